@@ -1,0 +1,374 @@
+// qsa_oracle.cpp -- plain, slow, float64 CPU oracle for the QSA sparse-attention step.
+//
+// TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+// call this file: only the tests, the smoke check and the bench's CPU-baseline
+// leg use it.  It shares no code, header, table or helper with the CUDA
+// library; both sides only see the same seeded inputs.
+//
+// What it computes (one query row at a time, never materialising T x L):
+//   1. indexer score of every visible cell c < V:
+//        score[c] = sum_h w[h] * max(0, sum_d iq[h][d] * key[c][d])       (4 heads x 64, fp16 in)
+//      The pages name the indexer ("indexer q" in "opus r20 track A ...",
+//      section 3; QSA's Wiq in "opus r15 track A ...", what changed, item 5)
+//      and its matrix form qsa_score_mm (same page, item 1) but print no
+//      formula; this is the workload's stated form, read plainly.
+//   2. top-k: the k visible cells of largest score, equal scores going to the
+//      lower cell index; every visible cell when V <= k; reported ascending,
+//      padded with -1.  One id set per token, shared by all heads (the qids
+//      row per token in "Round 5 Track C Report ...", section 1, Target 2).
+//   3. attention over the selected cells with int8 K/V and one fp16 scale per
+//      32 values ("random int8 KV, fp16 scales", "opus r20 track A ...",
+//      section 3): for head h (KV head g = h / 12),
+//        s_c = scale * sum_d q[h][d] * K[c][g][d] * ks[c][g][d/32]
+//        O   = sum_c exp(s_c - max s) * V[c][g][:] * vs[c][g][:/32] / sum_c exp(s_c - max s)
+//      (the max-subtracted softmax of qsa_attn, same page, section 2).
+//   4. split partials (m, l, o) over contiguous pieces of the selected list
+//      and their log-sum-exp merge M = max m_k, e_k = exp(m_k - M),
+//      L = sum l_k e_k, O = sum o_k e_k / L (qsa_merge, same page, section 2).
+//   5. the cache-write quantizer, per group of 32 fp32 values:
+//        amax = max |x|; s = fp16_rn(amax / 127 in fp32), saturated at 65504;
+//        q = clamp(rint(x / float(s)), -127, 127), all codes 0 when s == 0.
+//      The pages give only "int8 KV, fp16 scales"; the group of 32 and the
+//      rounding are the plainest reading.  The code is an integer decided by
+//      floating point, so the division and rounding are taken in fp32 exactly
+//      as the kernel takes them.
+//
+// Build: g++ -O2 -std=c++17 -fopenmp -shared -fPIC (see oracle/build.py).
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <limits>
+#include <vector>
+
+namespace {
+
+constexpr int kHQ = 24;       // query heads
+constexpr int kD = 256;       // head dim
+constexpr int kHKV = 2;       // KV heads
+constexpr int kGroup = 32;    // values per fp16 scale
+constexpr int kNG = kD / kGroup;
+constexpr int kHI = 4;        // indexer heads
+constexpr int kDI = 64;       // indexer dim
+constexpr int kQPerKV = kHQ / kHKV;
+
+// IEEE 754 binary16 -> double, written from the format's definition:
+// 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits.
+double half_to_double(uint16_t h) {
+  const int sign = h >> 15;
+  const int e = (h >> 10) & 0x1f;
+  const int f = h & 0x3ff;
+  double mag;
+  if (e == 0) {
+    mag = std::ldexp(static_cast<double>(f), -24);                 // subnormal: f * 2^-24
+  } else if (e == 31) {
+    mag = f ? std::numeric_limits<double>::quiet_NaN() : std::numeric_limits<double>::infinity();
+  } else {
+    mag = std::ldexp(static_cast<double>(1024 + f), e - 25);      // (1 + f/1024) * 2^(e-15)
+  }
+  return sign ? -mag : mag;
+}
+
+// Per-cell cache addressing: K/V rows [cell][kv head][256], scales [cell][kv head][8].
+struct CacheView {
+  const int8_t* k;
+  const int8_t* v;
+  const uint16_t* ks;
+  const uint16_t* vs;
+  const uint16_t* idx_key;
+};
+
+double k_deq(const CacheView& c, int64_t cell, int g, int d) {
+  return static_cast<double>(c.k[(cell * kHKV + g) * kD + d]) *
+         half_to_double(c.ks[(cell * kHKV + g) * kNG + d / kGroup]);
+}
+
+double v_deq(const CacheView& c, int64_t cell, int g, int d) {
+  return static_cast<double>(c.v[(cell * kHKV + g) * kD + d]) *
+         half_to_double(c.vs[(cell * kHKV + g) * kNG + d / kGroup]);
+}
+
+// Step 1 for one row over cells [0, V).
+void index_scores(const uint16_t* keys, int64_t V, const uint16_t* iq, const float* iw, double* out) {
+  for (int64_t c = 0; c < V; ++c) {
+    double s = 0.0;
+    for (int h = 0; h < kHI; ++h) {
+      double dot = 0.0;
+      for (int d = 0; d < kDI; ++d)
+        dot += half_to_double(iq[h * kDI + d]) * half_to_double(keys[c * kDI + d]);
+      s += static_cast<double>(iw[h]) * std::max(0.0, dot);
+    }
+    out[c] = s;
+  }
+}
+
+// Order of step 2: higher score first, then lower index.
+struct Before {
+  const double* s;
+  bool operator()(int32_t a, int32_t b) const {
+    if (s[a] != s[b]) return s[a] > s[b];
+    return a < b;
+  }
+};
+
+// Step 2: the first min(k, V) cells in the order above, reported ascending.
+int topk(const double* scores, int64_t V, int k, int32_t* ids) {
+  const int64_t take = std::min<int64_t>(k, V);
+  std::vector<int32_t> idx(static_cast<size_t>(V));
+  for (int64_t i = 0; i < V; ++i) idx[i] = static_cast<int32_t>(i);
+  if (take < V) std::nth_element(idx.begin(), idx.begin() + take, idx.end(), Before{scores});
+  idx.resize(static_cast<size_t>(take));
+  std::sort(idx.begin(), idx.end());
+  for (int64_t i = 0; i < take; ++i) ids[i] = idx[i];
+  for (int64_t i = take; i < k; ++i) ids[i] = -1;
+  return static_cast<int>(take);
+}
+
+// Step 3, one head: softmax attention over ids[0..count) (entries < 0 skipped).
+void attn_head(const CacheView& c, const float* qh, int g, const int32_t* ids, int count,
+               double scale, double* out) {
+  std::vector<double> s;
+  std::vector<int32_t> cells;
+  for (int i = 0; i < count; ++i) {
+    if (ids[i] < 0) continue;
+    double dot = 0.0;
+    for (int d = 0; d < kD; ++d) dot += static_cast<double>(qh[d]) * k_deq(c, ids[i], g, d);
+    s.push_back(scale * dot);
+    cells.push_back(ids[i]);
+  }
+  for (int d = 0; d < kD; ++d) out[d] = 0.0;
+  if (s.empty()) return;
+  const double m = *std::max_element(s.begin(), s.end());
+  double l = 0.0;
+  for (size_t j = 0; j < s.size(); ++j) {
+    const double p = std::exp(s[j] - m);
+    l += p;
+    for (int d = 0; d < kD; ++d) out[d] += p * v_deq(c, cells[j], g, d);
+  }
+  for (int d = 0; d < kD; ++d) out[d] /= l;
+}
+
+// Step 4, one head: partial (m, l, unnormalised o) over ids[0..count).
+// An empty piece gives m = -inf, l = 0, o = 0.
+void partial_head(const CacheView& c, const float* qh, int g, const int32_t* ids, int count,
+                  double scale, double* m_out, double* l_out, double* o) {
+  std::vector<double> s;
+  std::vector<int32_t> cells;
+  for (int i = 0; i < count; ++i) {
+    if (ids[i] < 0) continue;
+    double dot = 0.0;
+    for (int d = 0; d < kD; ++d) dot += static_cast<double>(qh[d]) * k_deq(c, ids[i], g, d);
+    s.push_back(scale * dot);
+    cells.push_back(ids[i]);
+  }
+  for (int d = 0; d < kD; ++d) o[d] = 0.0;
+  if (s.empty()) {
+    *m_out = -std::numeric_limits<double>::infinity();
+    *l_out = 0.0;
+    return;
+  }
+  const double m = *std::max_element(s.begin(), s.end());
+  double l = 0.0;
+  for (size_t j = 0; j < s.size(); ++j) {
+    const double p = std::exp(s[j] - m);
+    l += p;
+    for (int d = 0; d < kD; ++d) o[d] += p * v_deq(c, cells[j], g, d);
+  }
+  *m_out = m;
+  *l_out = l;
+}
+
+// Step 4, merge of nsplit partials for one head (pieces with l == 0 add nothing).
+void merge_head(const double* m, const double* l, const double* o, int nsplit, int stride_o,
+                double* out) {
+  double M = -std::numeric_limits<double>::infinity();
+  for (int j = 0; j < nsplit; ++j)
+    if (l[j] > 0.0) M = std::max(M, m[j]);
+  for (int d = 0; d < kD; ++d) out[d] = 0.0;
+  double L = 0.0;
+  for (int j = 0; j < nsplit; ++j) {
+    if (!(l[j] > 0.0)) continue;
+    const double e = std::exp(m[j] - M);
+    L += l[j] * e;
+    for (int d = 0; d < kD; ++d) out[d] += o[static_cast<size_t>(j) * stride_o + d] * e;
+  }
+  if (L > 0.0)
+    for (int d = 0; d < kD; ++d) out[d] /= L;
+}
+
+// Step 5 for one group of 32 values.
+void quantize_group(const float* x, int8_t* q, uint16_t* scale_bits) {
+  float amax = 0.0f;
+  for (int i = 0; i < kGroup; ++i) amax = std::max(amax, std::fabs(x[i]));
+  const float ratio = amax / 127.0f;
+  _Float16 sh = static_cast<_Float16>(ratio);
+  if (!(static_cast<float>(sh) <= 65504.0f)) sh = static_cast<_Float16>(65504.0f);
+  std::memcpy(scale_bits, &sh, sizeof(uint16_t));
+  const float sf = static_cast<float>(sh);
+  for (int i = 0; i < kGroup; ++i) {
+    if (sf == 0.0f) {
+      q[i] = 0;
+      continue;
+    }
+    const float r = std::nearbyint(x[i] / sf);
+    q[i] = static_cast<int8_t>(std::min(127.0f, std::max(-127.0f, r)));
+  }
+}
+
+// One full row: scores, selection, attention.  out [24][256]; ids [k];
+// scores_out (optional) [V].
+void row(const CacheView& c, int64_t V, const float* q, const uint16_t* iq, const float* iw, int k,
+         double scale, double* out, int32_t* ids, double* scores_out) {
+  std::vector<double> sc(static_cast<size_t>(V));
+  index_scores(c.idx_key, V, iq, iw, sc.data());
+  if (scores_out) std::copy(sc.begin(), sc.end(), scores_out);
+  topk(sc.data(), V, k, ids);
+  for (int h = 0; h < kHQ; ++h)
+    attn_head(c, q + static_cast<size_t>(h) * kD, h / kQPerKV, ids, k, scale,
+              out + static_cast<size_t>(h) * kD);
+}
+
+}  // namespace
+
+extern "C" {
+
+int qsa_oracle_version(void) { return 1; }
+
+double qsa_oracle_half_to_double(uint16_t h) { return half_to_double(h); }
+
+uint16_t qsa_oracle_float_to_half(float x) {
+  const _Float16 h = static_cast<_Float16>(x);
+  uint16_t b;
+  std::memcpy(&b, &h, sizeof(b));
+  return b;
+}
+
+void qsa_oracle_index_scores(const uint16_t* keys, int64_t V, const uint16_t* iq, const float* iw,
+                             double* out) {
+  index_scores(keys, V, iq, iw, out);
+}
+
+int qsa_oracle_topk(const double* scores, int64_t V, int k, int32_t* ids) {
+  return topk(scores, V, k, ids);
+}
+
+// Second, independent selector for the pins: a full stable sort of all V cells.
+int qsa_oracle_topk_fullsort(const double* scores, int64_t V, int k, int32_t* ids) {
+  std::vector<int32_t> idx(static_cast<size_t>(V));
+  for (int64_t i = 0; i < V; ++i) idx[i] = static_cast<int32_t>(i);
+  std::stable_sort(idx.begin(), idx.end(),
+                   [scores](int32_t a, int32_t b) { return scores[a] > scores[b]; });
+  const int64_t take = std::min<int64_t>(k, V);
+  std::vector<int32_t> top(idx.begin(), idx.begin() + take);
+  std::sort(top.begin(), top.end());
+  for (int64_t i = 0; i < take; ++i) ids[i] = top[i];
+  for (int64_t i = take; i < k; ++i) ids[i] = -1;
+  return static_cast<int>(take);
+}
+
+// Attention of one row (24 heads) over a given id list.
+void qsa_oracle_attn_row(const int8_t* k, const int8_t* v, const uint16_t* ks, const uint16_t* vs,
+                         const float* q, const int32_t* ids, int count, double scale, double* out) {
+  const CacheView c{k, v, ks, vs, nullptr};
+  for (int h = 0; h < kHQ; ++h)
+    attn_head(c, q + static_cast<size_t>(h) * kD, h / kQPerKV, ids, count, scale,
+              out + static_cast<size_t>(h) * kD);
+}
+
+// Partials of one row: the id list [0, count) cut into nsplit contiguous
+// pieces of ceil(count / nsplit) entries.  m, l: [24][nsplit]; o: [24][nsplit][256].
+void qsa_oracle_partials_row(const int8_t* k, const int8_t* v, const uint16_t* ks,
+                             const uint16_t* vs, const float* q, const int32_t* ids, int count,
+                             int nsplit, double scale, double* m, double* l, double* o) {
+  const CacheView c{k, v, ks, vs, nullptr};
+  const int piece = (count + nsplit - 1) / nsplit;
+  for (int h = 0; h < kHQ; ++h)
+    for (int j = 0; j < nsplit; ++j) {
+      const int b = std::min(count, j * piece), e = std::min(count, (j + 1) * piece);
+      const size_t hj = static_cast<size_t>(h) * nsplit + j;
+      partial_head(c, q + static_cast<size_t>(h) * kD, h / kQPerKV, ids + b, e - b, scale, m + hj,
+                   l + hj, o + hj * kD);
+    }
+}
+
+// Merge of one row: m, l [24][nsplit]; o [24][nsplit][256] -> out [24][256].
+void qsa_oracle_merge_row(const double* m, const double* l, const double* o, int nsplit,
+                          double* out) {
+  for (int h = 0; h < kHQ; ++h)
+    merge_head(m + static_cast<size_t>(h) * nsplit, l + static_cast<size_t>(h) * nsplit,
+               o + static_cast<size_t>(h) * nsplit * kD, nsplit, kD, out + static_cast<size_t>(h) * kD);
+}
+
+// Brute force: full softmax attention over every cell [0, V), no selection.
+void qsa_oracle_dense_attn_row(const int8_t* k, const int8_t* v, const uint16_t* ks,
+                               const uint16_t* vs, int64_t V, const float* q, double scale,
+                               double* out) {
+  for (int h = 0; h < kHQ; ++h) {
+    const int g = h / kQPerKV;
+    std::vector<double> s(static_cast<size_t>(V));
+    for (int64_t c = 0; c < V; ++c) {
+      double dot = 0.0;
+      for (int d = 0; d < kD; ++d) {
+        const double kd = static_cast<double>(k[(c * kHKV + g) * kD + d]) *
+                          half_to_double(ks[(c * kHKV + g) * kNG + d / kGroup]);
+        dot += static_cast<double>(q[h * kD + d]) * kd;
+      }
+      s[c] = scale * dot;
+    }
+    const double m = *std::max_element(s.begin(), s.end());
+    double den = 0.0;
+    std::vector<double> num(kD, 0.0);
+    for (int64_t c = 0; c < V; ++c) {
+      const double p = std::exp(s[c] - m);
+      den += p;
+      for (int d = 0; d < kD; ++d)
+        num[d] += p * static_cast<double>(v[(c * kHKV + g) * kD + d]) *
+                  half_to_double(vs[(c * kHKV + g) * kNG + d / kGroup]);
+    }
+    for (int d = 0; d < kD; ++d) out[h * kD + d] = num[d] / den;
+  }
+}
+
+// Quantizer over ngroups groups of 32 values.
+void qsa_oracle_quantize(const float* x, int64_t ngroups, int8_t* q, uint16_t* scale_bits) {
+  for (int64_t i = 0; i < ngroups; ++i) quantize_group(x + i * kGroup, q + i * kGroup, scale_bits + i);
+}
+
+// Cache write: quantize n cells of fp32 K/V [n][2][256] into the cache at
+// cells pos0..pos0+n-1 and copy their fp16 indexer keys [n][64].
+void qsa_oracle_cache_write(int8_t* kc, int8_t* vc, uint16_t* ks, uint16_t* vs, uint16_t* idx_key,
+                            int64_t pos0, int n, const float* k, const float* v,
+                            const uint16_t* key) {
+  for (int i = 0; i < n; ++i) {
+    const int64_t cell = pos0 + i;
+    for (int g = 0; g < kHKV; ++g)
+      for (int j = 0; j < kNG; ++j) {
+        const size_t src = (static_cast<size_t>(i) * kHKV + g) * kD + j * kGroup;
+        const size_t dst = (static_cast<size_t>(cell) * kHKV + g) * kD + j * kGroup;
+        const size_t sdst = (static_cast<size_t>(cell) * kHKV + g) * kNG + j;
+        quantize_group(k + src, kc + dst, ks + sdst);
+        quantize_group(v + src, vc + dst, vs + sdst);
+      }
+    std::memcpy(idx_key + cell * kDI, key + static_cast<size_t>(i) * kDI, kDI * sizeof(uint16_t));
+  }
+}
+
+// Rows rows[0..nrows) of one call; row r sees vis0 + r cells.  out [nrows][24][256],
+// ids [nrows][k], scores (optional) [nrows][vmax] with vmax = vis0 + max row.
+// Rows run in parallel over the host cores (independent by definition).
+void qsa_oracle_rows(const int8_t* k, const int8_t* v, const uint16_t* ks, const uint16_t* vs,
+                     const uint16_t* idx_key, int64_t vis0, const int32_t* rows, int nrows,
+                     const float* q, const uint16_t* iq, const float* iw, int top_k, double scale,
+                     double* out, int32_t* ids, double* scores, int64_t ld_scores, int threads) {
+  const CacheView c{k, v, ks, vs, idx_key};
+#pragma omp parallel for schedule(dynamic, 1) num_threads(threads > 0 ? threads : 1)
+  for (int i = 0; i < nrows; ++i) {
+    const int r = rows[i];
+    row(c, vis0 + r, q + static_cast<size_t>(r) * kHQ * kD, iq + static_cast<size_t>(r) * kHI * kDI,
+        iw + static_cast<size_t>(r) * kHI, top_k, scale, out + static_cast<size_t>(i) * kHQ * kD,
+        ids + static_cast<size_t>(i) * top_k,
+        scores ? scores + static_cast<size_t>(i) * ld_scores : nullptr);
+  }
+}
+
+}  // extern "C"
