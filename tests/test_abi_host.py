@@ -1,0 +1,106 @@
+"""Host-side checks of the C ABI: the library builds, loads and exports every
+entry point of include/qsa.h, and rejects bad arguments before touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import torch  # noqa: F401  (loads the CUDA runtime the library links against)
+    from top_sparse_attention_score_b200 import build, qsa
+    build.build()
+    return qsa.load()
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(qsa_\w+)\s*\(", src, flags=re.M)
+    return names
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    for n in ["qsa_workspace_bytes", "qsa_cache_write", "qsa_decode", "qsa_prefill_chunk",
+              "qsa_index_score", "qsa_topk_workspace_bytes", "qsa_topk", "qsa_attn", "qsa_merge",
+              "qsa_last_error", "qsa_launch_count"]:
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    from top_sparse_attention_score_b200 import qsa
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert name in qsa.SIGNATURES, f"binding lacks a signature for {name}"
+
+
+def _fake_cache(qsa, cells=1000):
+    # Aligned, non-NULL host addresses: only used by calls that must fail validation.
+    return qsa.CacheStruct(0x10000, 0x20000, 0x30000, 0x40000, 0x50000, cells)
+
+
+def test_workspace_bytes(lib):
+    assert lib.qsa_workspace_bytes(0, 0, 100, 10, 0) == 0
+    assert lib.qsa_workspace_bytes(0, 9, 100, 10, 0) == 0          # n > 8
+    assert lib.qsa_workspace_bytes(0, 1, 100, 0, 0) == 0           # top_k < 1
+    assert lib.qsa_workspace_bytes(0, 1, 100, 10, 65) == 0         # nsplit > 64
+    assert lib.qsa_workspace_bytes(2, 1, 100, 10, 0) == 0          # bad mode
+    a = lib.qsa_workspace_bytes(0, 1, 4096, 512, 1)
+    b = lib.qsa_workspace_bytes(0, 1, 65536, 512, 1)
+    c = lib.qsa_workspace_bytes(0, 1, 65536, 512, 64)
+    assert 0 < a < b < c
+    # scores alone need rows * L * 4 bytes
+    assert lib.qsa_workspace_bytes(1, 1024, 262144, 2048, 0) >= 1024 * 262144 * 4
+    assert lib.qsa_topk_workspace_bytes(4, 1000, 100) > 4 * 2048 * 4
+
+
+def test_decode_rejects_bad_arguments(lib):
+    from top_sparse_attention_score_b200 import qsa
+    cs = _fake_cache(qsa)
+    P = ctypes.c_void_p(0x60000)
+    def call(L=1000, n=1, top_k=64, nsplit=0, ws_bytes=1 << 40, q=P, cache=ctypes.byref(cs)):
+        return lib.qsa_decode(cache, L, n, q, P, P, top_k, nsplit, 0.0625, P, ws_bytes, P, None, None)
+    assert call(n=0) == 1 and "n = 0" in qsa.last_error()
+    assert call(n=9) == 1
+    assert call(L=1001) == 1                      # beyond max_cells
+    assert call(L=2, n=3) == 1                    # L < n
+    assert call(top_k=0) == 1
+    assert call(top_k=16385) == 1
+    assert call(nsplit=65) == 1
+    assert call(q=None) == 1
+    assert call(q=ctypes.c_void_p(0x60004)) == 1  # misaligned
+    assert call(ws_bytes=100) == 2 and "workspace" in qsa.last_error()
+    assert call(cache=None) == 1
+    bad = qsa.CacheStruct(0x10000, 0, 0x30000, 0x40000, 0x50000, 1000)
+    assert call(cache=ctypes.byref(bad)) == 1
+
+
+def test_prefill_and_steps_reject_bad_arguments(lib):
+    from top_sparse_attention_score_b200 import qsa
+    cs = _fake_cache(qsa)
+    P = ctypes.c_void_p(0x60000)
+    cb = ctypes.byref(cs)
+    assert lib.qsa_prefill_chunk(cb, 990, 20, P, P, P, 64, 0.0625, P, 1 << 40, P, None, None) == 1
+    assert lib.qsa_prefill_chunk(cb, -1, 20, P, P, P, 64, 0.0625, P, 1 << 40, P, None, None) == 1
+    assert lib.qsa_prefill_chunk(cb, 0, 20, P, P, P, 64, 0.0625, P, 10, P, None, None) == 2
+    assert lib.qsa_cache_write(cb, 999, 2, P, P, P, None) == 1
+    assert lib.qsa_cache_write(cb, 0, 0, P, P, P, None) == 1
+    assert lib.qsa_index_score(cb, 1, 100, P, P, P, 99, None) == 1       # ld < ncells
+    assert lib.qsa_index_score(cb, 1, 100, P, P, P, 102, None) == 1      # ld % 4
+    assert lib.qsa_index_score(cb, 1, 1001, P, P, P, 1004, None) == 1    # ncells > max_cells
+    assert lib.qsa_topk(P, 100, 2, 100, 10, P, 1 << 40, P, None) == 1    # row 1 sees 101 > ld
+    assert lib.qsa_topk(P, 100, 1, 0, 10, P, 1 << 40, P, None) == 1      # vis0 < 1
+    assert lib.qsa_topk(P, 100, 1, 50, 10, P, 10, P, None) == 2
+    assert lib.qsa_attn(cb, 1, P, P, 64, 0, 0.0625, P, P, None) == 1
+    assert lib.qsa_attn(cb, 1, P, P, 64, 2, 0.0625, None, P, None) == 1  # nsplit > 1 needs part
+    assert lib.qsa_attn(cb, 1, P, P, 64, 1, 0.0625, P, None, None) == 1  # nsplit 1 needs out
+    assert lib.qsa_merge(None, 1, 2, P, None) == 1
+    assert lib.qsa_merge(P, 1, 65, P, None) == 1

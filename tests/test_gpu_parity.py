@@ -1,0 +1,444 @@
+"""CUDA path against the CPU oracle on the same seeded inputs (needs a B200).
+
+Tolerances (fixed by the workload statement):
+* selected id sets are bit-exact, except that a cell may be swapped at the
+  k-th boundary when its oracle score is within 1e-5 relative of the oracle's
+  k-th score tau (GPU scores are fp32, the oracle's float64);
+* attention outputs are within 2e-3 relative error, measured per (row, head)
+  as max_d |O_gpu - O_ref| / max_d |O_ref|;
+* the cache-write codes and scales, and the selection on identical fp32
+  scores, are bit-exact.
+"""
+from __future__ import annotations
+
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+OUT_TOL = 2e-3
+SEL_TOL = 1e-5
+SPLIT_TOL = 1e-3   # GPU against GPU with a different split of the selected list
+THREADS = os.cpu_count() or 1
+
+
+def dev_inputs(qsa, wl):
+    cache = qsa.DeviceCache.from_host(wl.cache, DEV)
+    return (cache, torch.from_numpy(wl.q).to(DEV), torch.from_numpy(wl.iq).to(DEV),
+            torch.from_numpy(wl.iw).to(DEV))
+
+
+def rel_err(out, ref):
+    """max over (row, head) of max_d |out - ref| / max_d |ref|."""
+    den = np.maximum(np.abs(ref).max(-1), 1e-30)
+    return float((np.abs(out - ref).max(-1) / den).max())
+
+
+def check_selection(ids, ref_ids, ref_scores, top_k):
+    """Apply the boundary rule row by row; return the rows whose sets match exactly."""
+    exact = []
+    for r in range(ref_ids.shape[0]):
+        g = ids[r]
+        o = ref_ids[r]
+        nv = int((o >= 0).sum())
+        assert int((g >= 0).sum()) == nv, f"row {r}: {int((g >= 0).sum())} ids, oracle {nv}"
+        assert np.all(g[nv:] == -1) and np.all(np.diff(g[:nv]) > 0), f"row {r}: not ascending / padded"
+        gs, os_ = set(g[:nv].tolist()), set(o[:nv].tolist())
+        if gs == os_:
+            exact.append(r)
+            continue
+        tau = ref_scores[r][o[:nv]].min()
+        for c in gs ^ os_:
+            assert abs(ref_scores[r][c] - tau) <= SEL_TOL * abs(tau), (
+                f"row {r}: cell {c} (score {ref_scores[r][c]!r}) differs beyond the boundary tau={tau!r}")
+    return exact
+
+
+def check_outputs(qsa, cache, q, out, ids, ref_out, ref_ids, ref_scores, rows, scale, top_k):
+    exact = set(check_selection(ids, ref_ids, ref_scores, top_k))
+    for i, r in enumerate(rows):
+        if i in exact:
+            e = rel_err(out[r], ref_out[i])
+        else:  # boundary swap: run the GPU attention on the oracle's own selection
+            o2 = qsa.attn(cache, q[r:r + 1].contiguous(),
+                          torch.from_numpy(ref_ids[i:i + 1]).to(DEV), 1, scale)
+            e = rel_err(o2.cpu().numpy()[0], ref_out[i])
+        assert e <= OUT_TOL, f"row {r}: relative error {e:.3e}"
+    return len(exact)
+
+
+# ------------------------------------------------------------------ cache write
+
+@pytest.mark.parametrize("pattern", ["random", "signed_zeros", "pow2", "alternating", "tiny"])
+def test_cache_write_bit_exact(gpu, pattern):
+    qsa = gpu
+    cells, pos0, n = 40, 13, 7
+    host = synth.make_cache(5, cells)
+    x = synth.quantizer_patterns(17, 2 * n * 2 * 8)[pattern].reshape(2, n, 2, 256)
+    key = synth.make_new_cells(18, n)[2]
+    cache = qsa.DeviceCache.from_host(host, DEV)
+    qsa.cache_write(cache, pos0, torch.from_numpy(np.ascontiguousarray(x[0])).to(DEV),
+                    torch.from_numpy(np.ascontiguousarray(x[1])).to(DEV), torch.from_numpy(key).to(DEV))
+    oracle.cache_write(host, pos0, x[0], x[1], key)
+    torch.cuda.synchronize()
+    assert np.array_equal(cache.k.cpu().numpy(), host.k)
+    assert np.array_equal(cache.v.cpu().numpy(), host.v)
+    assert np.array_equal(cache.ks.cpu().numpy().view(np.uint16), host.ks.view(np.uint16))
+    assert np.array_equal(cache.vs.cpu().numpy().view(np.uint16), host.vs.view(np.uint16))
+    assert np.array_equal(cache.idx_key.cpu().numpy().view(np.uint16), host.idx_key.view(np.uint16))
+
+
+def test_cache_write_golden(gpu):
+    """The hand-worked quantizer fixtures, through the kernel."""
+    from tests import pins
+    qsa = gpu
+    cases = pins.load_quantize_golden()
+    n = (len(cases) + 15) // 16
+    x = np.zeros((n * 16, 32), np.float32)
+    for i, (_, xi, _, _) in enumerate(cases):
+        x[i] = xi
+    cache = qsa.DeviceCache.empty(n, DEV)
+    xk = torch.from_numpy(x.reshape(n, 2, 256)).to(DEV)
+    qsa.cache_write(cache, 0, xk, xk, torch.zeros(n, 64, dtype=torch.float16, device=DEV))
+    codes = cache.k.cpu().numpy().reshape(-1, 32)
+    scales = cache.ks.cpu().numpy().view(np.uint16).reshape(-1)
+    for i, (name, _, sbits, want) in enumerate(cases):
+        assert int(scales[i]) == sbits, name
+        assert np.array_equal(codes[i], want), name
+
+
+# ------------------------------------------------------------------ index score
+
+@pytest.mark.parametrize("ncells,rows", [(1000, 8), (77, 3), (4096, 1), (333, 13)])
+def test_index_score(gpu, ncells, rows):
+    qsa = gpu
+    wl = synth.make_workload(1, n=min(rows, 8), cells=ncells)
+    _, iq, iw = synth.make_queries(77, rows)
+    cache = qsa.DeviceCache.from_host(wl.cache, DEV)
+    sc = qsa.index_score(cache, torch.from_numpy(iq).to(DEV), torch.from_numpy(iw).to(DEV), ncells)
+    torch.cuda.synchronize()
+    sc = sc.cpu().numpy()[:, :ncells]
+    key = wl.cache.idx_key.astype(np.float64)
+    for r in range(rows):
+        ref = oracle.index_scores(wl.cache.idx_key, ncells, iq[r], iw[r])
+        # fp32 accumulation of 64 exact fp16 products: at most 64 ulps of the sum of |terms|
+        terms = np.abs(iq[r].astype(np.float64)) @ np.abs(key).T          # [4][ncells]
+        bound = 2.0 ** -18 * (iw[r].astype(np.float64) @ terms) + 1e-30
+        err = np.abs(sc[r] - ref)
+        assert np.all(err <= bound), (r, float((err / bound).max()))
+
+
+def test_index_score_duplicates_bit_equal(gpu):
+    qsa = gpu
+    wl = synth.make_workload(4, cells=3000, rows=4)
+    cache = qsa.DeviceCache.from_host(wl.cache, DEV)
+    sc = qsa.index_score(cache, torch.from_numpy(wl.iq).to(DEV), torch.from_numpy(wl.iw).to(DEV), 3000)
+    sc = sc.cpu().numpy()[:, :3000]
+    keys = wl.cache.idx_key.view(np.uint16)
+    _, first = np.unique(keys, axis=0, return_index=True)
+    inv = np.unique(keys, axis=0, return_inverse=True)[1].reshape(-1)
+    assert first.size < 3000  # the workload has duplicates
+    for r in range(4):
+        assert np.array_equal(sc[r], sc[r][first[inv]])
+
+
+# ------------------------------------------------------------------ selection
+
+def _topk_case(qsa, scores, vis0, k):
+    rows = scores.shape[0]
+    ld = (scores.shape[1] + 3) // 4 * 4
+    s = np.zeros((rows, ld), np.float32)
+    s[:, :scores.shape[1]] = scores
+    ids = qsa.topk(torch.from_numpy(s).to(DEV), vis0, k).cpu().numpy()
+    for r in range(rows):
+        ref = oracle.topk(scores[r, :vis0 + r].astype(np.float64), k)
+        assert np.array_equal(ids[r], ref), (r, np.setdiff1d(ids[r], ref)[:5], np.setdiff1d(ref, ids[r])[:5])
+
+
+def test_topk_random(gpu):
+    st = synth.Stream(101, "tk")
+    _topk_case(gpu, st.normal(3 * 5003).astype(np.float32).reshape(3, 5003), 5001, 512)
+
+
+def test_topk_ties(gpu):
+    st = synth.Stream(102, "tk")
+    s = (np.round(st.normal(2 * 20000) * 2) / 2).astype(np.float32).reshape(2, 20000)
+    _topk_case(gpu, s, 19999, 2048)
+
+
+@pytest.mark.parametrize("V,k", [(100, 512), (512, 512), (513, 512), (1, 1), (40, 1), (4097, 4096)])
+def test_topk_sizes(gpu, V, k):
+    st = synth.Stream(103 + V, "tk")
+    s = st.normal(2 * (V + 1)).astype(np.float32).reshape(2, V + 1)
+    _topk_case(gpu, s, V, k)
+
+
+def test_topk_all_equal_and_signed_zero(gpu):
+    s = np.zeros((2, 3000), np.float32)
+    s[1, ::2] = -0.0
+    s[1, 5] = -1e-30
+    _topk_case(gpu, s, 2999, 700)
+
+
+def test_topk_negative(gpu):
+    st = synth.Stream(104, "tk")
+    _topk_case(gpu, (-np.abs(st.normal(2 * 9000)) - 3).astype(np.float32).reshape(2, 9000), 8999, 1000)
+
+
+def test_topk_candidate_overflow(gpu):
+    # every score in one coarse (fp16) bin, all distinct in fp32: the candidate list
+    # overflows and the final pass re-reads the row
+    st = synth.Stream(105, "tk")
+    V = 50000
+    s = (1.0 + np.floor(st.uniform(V) * 4096) * 2.0 ** -23).astype(np.float32)[None, :]
+    _topk_case(gpu, s, V, 2048)
+
+
+def test_topk_many_windows(gpu):
+    st = synth.Stream(106, "tk")
+    V = (1 << 19) * 2 + 777
+    s = np.round(st.normal(V) * 64).astype(np.float32)[None, :]
+    _topk_case(gpu, s, V, 4096)
+
+
+def test_topk_max_k(gpu):
+    st = synth.Stream(107, "tk")
+    _topk_case(gpu, st.normal(40000).astype(np.float32)[None, :], 40000, 16384)
+
+
+# ------------------------------------------------------------------ attention and merge
+
+def _id_lists(seed, rows, cells, k, nvalid):
+    st = synth.Stream(seed, "ids")
+    ids = -np.ones((rows, k), np.int32)
+    for r in range(rows):
+        pick = np.sort(np.argsort(st.uniform(cells), kind="stable")[:nvalid[r]]).astype(np.int32)
+        ids[r, :nvalid[r]] = pick
+    return ids
+
+
+@pytest.mark.parametrize("nsplit", [1, 3, 8, 64])
+def test_attn_vs_oracle(gpu, nsplit):
+    qsa = gpu
+    cells, k = 4096, 512
+    wl = synth.make_workload(0, cells=cells)
+    q, _, _ = synth.make_queries(201, 3)
+    ids = _id_lists(202, 3, cells, k, [512, 300, 17])
+    cache = qsa.DeviceCache.from_host(wl.cache, DEV)
+    qd = torch.from_numpy(q).to(DEV)
+    idd = torch.from_numpy(ids).to(DEV)
+    res = qsa.attn(cache, qd, idd, nsplit, 1 / 16)
+    out = res if nsplit == 1 else qsa.merge(res)
+    torch.cuda.synchronize()
+    out = out.cpu().numpy()
+    for r in range(3):
+        ref = oracle.attn_row(wl.cache, q[r], ids[r], 1 / 16)
+        assert rel_err(out[r], ref) <= OUT_TOL
+    if nsplit > 1:
+        part = res.cpu().numpy()
+        for r in range(3):
+            m, l, o = oracle.partials_row(wl.cache, q[r], ids[r], nsplit, 1 / 16)
+            pm, pl, po = part[r, :, :, 0], part[r, :, :, 1], part[r, :, :, 2:].astype(np.float64)
+            empty = l == 0
+            assert np.array_equal(pl == 0, empty) and np.all(np.isneginf(pm[empty]))
+            assert np.all(po[empty] == 0)
+            full = ~empty
+            # the piece maximum (natural-log units), its sum of weights, and its own output o / l
+            assert np.all(np.abs(pm[full] - m[full]) <= 2e-3)
+            assert np.allclose(pl[full] * np.exp(pm[full] - m[full]), l[full], rtol=5e-3)
+            assert rel_err(po[full] / pl[full][:, None], o[full] / l[full][:, None]) <= OUT_TOL
+
+
+def test_attn_small_v_scales(gpu):
+    qsa = gpu
+    cells = 2000
+    cache_h = synth.make_cache(203, cells, vs_range=(1e-4, 0.05))
+    q, _, _ = synth.make_queries(204, 2)
+    ids = _id_lists(205, 2, cells, 2048, [2000, 1999])
+    cache = qsa.DeviceCache.from_host(cache_h, DEV)
+    out = qsa.attn(cache, torch.from_numpy(q).to(DEV), torch.from_numpy(ids).to(DEV), 1, 1 / 16).cpu().numpy()
+    for r in range(2):
+        assert rel_err(out[r], oracle.attn_row(cache_h, q[r], ids[r], 1 / 16)) <= OUT_TOL
+
+
+def test_attn_single_and_empty(gpu):
+    qsa = gpu
+    cache_h = synth.make_cache(206, 64)
+    q, _, _ = synth.make_queries(207, 2)
+    ids = -np.ones((2, 40), np.int32)
+    ids[0, 0] = 37  # one cell: O = its dequantised V row
+    cache = qsa.DeviceCache.from_host(cache_h, DEV)
+    out = qsa.attn(cache, torch.from_numpy(q).to(DEV), torch.from_numpy(ids).to(DEV), 1).cpu().numpy()
+    vd = cache_h.v[37].astype(np.float64) * np.repeat(cache_h.vs[37].astype(np.float64), 32, -1)
+    for h in range(24):
+        assert np.allclose(out[0, h], vd[h // 12], rtol=1e-3, atol=0)
+    assert np.all(out[1] == 0)  # no cells at all
+    part = qsa.attn(cache, torch.from_numpy(q).to(DEV), torch.from_numpy(ids).to(DEV), 4).cpu().numpy()
+    assert np.all(np.isneginf(part[1, :, :, 0])) and np.all(part[1, :, :, 1:] == 0)
+
+
+def test_merge_vs_oracle(gpu):
+    qsa = gpu
+    st = synth.Stream(301, "merge")
+    rows, ns = 3, 64
+    m = st.normal(rows * 24 * ns).reshape(rows, 24, ns) * 3
+    l = st.uniform(rows * 24 * ns, 0.5, 100).reshape(rows, 24, ns)
+    o = st.normal(rows * 24 * ns * 256).reshape(rows, 24, ns, 256) * 10
+    empty = st.uniform(rows * 24 * ns).reshape(rows, 24, ns) < 0.2
+    m[empty], l[empty], o[empty] = -np.inf, 0, 0
+    part = np.concatenate([m[..., None], l[..., None], o], -1).astype(np.float32)
+    out = qsa.merge(torch.from_numpy(part).to(DEV)).cpu().numpy()
+    for r in range(rows):
+        ref = oracle.merge_row(part[r, :, :, 0].astype(np.float64), part[r, :, :, 1].astype(np.float64),
+                               part[r, :, :, 2:].astype(np.float64))
+        assert rel_err(out[r], ref) <= 1e-5
+
+
+def test_merge_golden(gpu):
+    qsa = gpu
+    from tests import pins
+    import os as _os
+    lines = [ln for ln in open(_os.path.join(pins.GOLDEN, "merge_hand.txt")) if ln.startswith("case ")]
+    for ln in lines:
+        parts = [p.strip() for p in ln.split("|")]
+        m = np.array([float(t) for t in parts[1].split()[1:]])
+        l = np.array([float(t) for t in parts[2].split()[1:]])
+        o = np.array([float(t) for t in parts[3].split()[1:]])
+        want = float(parts[4].split()[1])
+        ns = m.size
+        part = np.zeros((1, 24, ns, 258), np.float32)
+        part[0, :, :, 0], part[0, :, :, 1] = m, l
+        part[0, :, :, 2:] = o[None, :, None] * np.arange(1, 257)[None, None, :]
+        out = qsa.merge(torch.from_numpy(part).to(DEV)).cpu().numpy()
+        assert np.allclose(out[0], want * np.arange(1, 257)[None, :], rtol=2e-6), parts[0]
+
+
+# ------------------------------------------------------------------ the whole step
+
+def _decode_case(qsa, wl, nsplit=None):
+    cache, q, iq, iw = dev_inputs(qsa, wl)
+    ids = torch.empty(wl.rows, wl.top_k, dtype=torch.int32, device=DEV)
+    ns = wl.nsplit if nsplit is None else nsplit
+    out = qsa.decode(cache, wl.L, q, iq, iw, wl.top_k, ns, wl.scale, ids_out=ids)
+    torch.cuda.synchronize()
+    ref_out, ref_ids, ref_sc = oracle.rows(wl, want_scores=True, threads=THREADS)
+    return check_outputs(qsa, cache, q, out.cpu().numpy(), ids.cpu().numpy(), ref_out, ref_ids, ref_sc,
+                         list(range(wl.rows)), wl.scale, wl.top_k)
+
+
+def test_decode_config0(gpu):
+    assert _decode_case(gpu, synth.make_workload(0)) >= 0
+
+
+@pytest.mark.parametrize("nsplit", [1, 8])
+def test_decode_config0_splits(gpu, nsplit):
+    _decode_case(gpu, synth.make_workload(0), nsplit)
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 4, 5, 6, 7, 8])
+def test_decode_config1(gpu, n):
+    _decode_case(gpu, synth.make_workload(1, n=n))
+
+
+def test_decode_config2(gpu):
+    _decode_case(gpu, synth.make_workload(2))
+
+
+def test_decode_small_ragged(gpu):
+    wl = synth.make_workload(1, n=5, cells=2077)
+    wl.top_k = 300
+    _decode_case(gpu, wl, 7)
+
+
+def test_decode_dense_when_few_cells(gpu):
+    # every row sees fewer cells than top_k: all visible cells, equal to brute-force softmax
+    qsa = gpu
+    wl = synth.make_workload(1, n=4, cells=300)
+    wl.top_k = 512
+    cache, q, iq, iw = dev_inputs(qsa, wl)
+    ids = torch.empty(4, 512, dtype=torch.int32, device=DEV)
+    out = qsa.decode(cache, wl.L, q, iq, iw, 512, 0, wl.scale, ids_out=ids).cpu().numpy()
+    ids = ids.cpu().numpy()
+    for i in range(4):
+        V = wl.L - 4 + 1 + i
+        assert np.array_equal(ids[i, :V], np.arange(V)) and np.all(ids[i, V:] == -1)
+        assert rel_err(out[i], oracle.dense_attn_row(wl.cache, V, wl.q[i], wl.scale)) <= OUT_TOL
+
+
+def test_decode_nsplit_invariance(gpu):
+    qsa = gpu
+    wl = synth.make_workload(1, n=2, cells=6000)
+    cache, q, iq, iw = dev_inputs(qsa, wl)
+    outs, idss = [], []
+    for ns in (1, 2, 7, 64):
+        ids = torch.empty(2, wl.top_k, dtype=torch.int32, device=DEV)
+        outs.append(qsa.decode(cache, wl.L, q, iq, iw, wl.top_k, ns, wl.scale, ids_out=ids).cpu().numpy())
+        idss.append(ids.cpu().numpy())
+    # Q and the softmax weights P are rounded to fp16 relative to each piece's own
+    # running maximum, so split counts differ by that rounding (~2^-12 relative per
+    # weight), well inside the parity tolerance each of them meets against the oracle.
+    for o, i in zip(outs[1:], idss[1:]):
+        assert np.array_equal(i, idss[0])
+        assert rel_err(o, outs[0]) <= SPLIT_TOL
+
+
+def _prefill_case(qsa, wl, rows):
+    cache, q, iq, iw = dev_inputs(qsa, wl)
+    ids = torch.empty(wl.rows, wl.top_k, dtype=torch.int32, device=DEV)
+    out = qsa.prefill_chunk(cache, wl.pos0, q, iq, iw, wl.top_k, wl.scale, ids_out=ids)
+    torch.cuda.synchronize()
+    ref_out, ref_ids, ref_sc = oracle.rows(wl, np.array(rows), want_scores=True, threads=THREADS)
+    return check_outputs(qsa, cache, q, out.cpu().numpy(), ids.cpu().numpy()[rows], ref_out, ref_ids,
+                         ref_sc, rows, wl.scale, wl.top_k)
+
+
+def test_prefill_small_all_rows(gpu):
+    wl = synth.make_workload(3, cells=2500, rows=150)
+    wl.top_k = 256
+    _prefill_case(gpu, wl, list(range(150)))
+
+
+def test_prefill_config3_sampled(gpu):
+    wl = synth.make_workload(3)
+    _prefill_case(gpu, wl, [0, 1, 777, 1500, 2046, 2047])
+
+
+def test_prefill_config4_sampled(gpu):
+    wl = synth.make_workload(4)
+    _prefill_case(gpu, wl, [0, 511, 1022, 1023])
+
+
+def test_prefill_row_equals_decode(gpu):
+    # prefill row t is a one-token decode at L = pos0 + t + 1 (both GPU paths)
+    qsa = gpu
+    wl = synth.make_workload(3, cells=3000, rows=64)
+    wl.top_k = 512
+    cache, q, iq, iw = dev_inputs(qsa, wl)
+    ids_p = torch.empty(64, 512, dtype=torch.int32, device=DEV)
+    out_p = qsa.prefill_chunk(cache, wl.pos0, q, iq, iw, 512, wl.scale, ids_out=ids_p)
+    for t in (0, 31, 63):
+        ids_d = torch.empty(1, 512, dtype=torch.int32, device=DEV)
+        out_d = qsa.decode(cache, wl.pos0 + t + 1, q[t:t + 1], iq[t:t + 1], iw[t:t + 1], 512, 1, wl.scale,
+                           ids_out=ids_d)
+        assert torch.equal(ids_d[0], ids_p[t])
+        # prefill picks its own split count; see test_decode_nsplit_invariance
+        assert rel_err(out_d.cpu().numpy()[0], out_p.cpu().numpy()[t]) <= SPLIT_TOL
+
+
+def test_errors_and_launch_count(gpu):
+    qsa = gpu
+    wl = synth.make_workload(0, cells=500)
+    cache, q, iq, iw = dev_inputs(qsa, wl)
+    small = qsa.workspace(64, DEV)
+    before = qsa.launch_count()
+    with pytest.raises(qsa.QSAError) as e:
+        qsa.decode(cache, wl.L, q, iq, iw, wl.top_k, 0, wl.scale, ws=small)
+    assert e.value.code == 2 and qsa.launch_count() == before
+    qsa.decode(cache, wl.L, q, iq, iw, wl.top_k, 0, wl.scale)
+    assert qsa.launch_count() > before

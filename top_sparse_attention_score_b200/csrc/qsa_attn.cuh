@@ -1,0 +1,304 @@
+// qsa_attn.cuh -- sparse attention over the selected cells of an int8 K/V cache.
+//
+// qsa_attn of "opus r20 track A: MTP map mlock + qsa_attn / qsa_merge decode tweaks",
+// section 2 (max-subtracted softmax over the selected cells, then a weighted sum of V),
+// on "random int8 KV, fp16 scales" (section 3), written for sm_100a:
+//
+//  * one CTA per (row, KV head, split); the 12 query heads of the KV head are the
+//    16 rows of mma.sync m16n8k16 tiles (rows 12..15 zero), so QK^T and PV run on
+//    tensor cores instead of 6144 fp32 FMAs per gathered cell;
+//  * cells are gathered 32 at a time with cp.async (16-byte copies of whole
+//    256-byte K/V rows and their scales) into a double-buffered shared-memory
+//    stage, so the next block's gathers are in flight while this one computes;
+//  * the four warps split the 256 dims: each computes a partial QK^T over its
+//    64 dims (two scale groups), the partials are summed through shared memory
+//    in a fixed order (all warps get bit-equal scores), each warp runs the same
+//    online softmax and accumulates P.V for its own 64 dims;
+//  * int8 codes become fp16 exactly (byte-permute with the 0x6400 exponent).  The
+//    per-32 K scale multiplies each 32-dim partial product in fp32 after the
+//    MMA; the per-32 V scale multiplies the fp16 V operand.  Q and P are fp16.
+#pragma once
+
+#include "qsa_common.cuh"
+
+namespace qsa {
+
+constexpr int kAttnCells = 32;    // cells per pipeline block
+constexpr int kAttnKStride = 288; // bytes per K row in shared memory (72 words: conflict-free 8-byte reads)
+constexpr int kAttnVStride = 272; // bytes per V row in shared memory (68 words: conflict-free 4-byte reads)
+
+struct __align__(16) AttnStage {
+  int8_t k[kAttnCells * kAttnKStride];
+  int8_t v[kAttnCells * kAttnVStride];
+  __half ks[kAttnCells * kNG];
+  __half vs[kAttnCells * kNG];
+  int valid[kAttnCells];
+};
+
+struct AttnSmem {
+  AttnStage st[2];
+  float4 red[4][4][32];  // [warp][n-tile][lane] partial scores
+};
+
+struct AttnArgs {
+  const int8_t* k;
+  const int8_t* v;
+  const __half* ks;
+  const __half* vs;
+  const float* q;     // [rows][24][256]
+  const int* ids;     // [rows][top_k]
+  int top_k;
+  int max_cells;      // ids outside [0, max_cells) are treated as empty slots
+  int nsplit;
+  int piece;          // ceil(top_k / nsplit)
+  float scale_log2;   // softmax scale * log2(e)
+  float* part;        // [rows][24][nsplit][258] when nsplit > 1
+  float* out;         // [rows][24][256] when nsplit == 1
+};
+
+__device__ __forceinline__ void attn_issue(AttnStage& st, const AttnArgs& a, const int* rid, int pos0,
+                                           int end, int kvh) {
+  const int tid = threadIdx.x;
+  // K and V rows: 32 cells x 16 chunks of 16 bytes each, 4 + 4 per thread.
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int chunk = tid + 128 * u;
+    const int i = chunk >> 4, part = chunk & 15;
+    const int p = pos0 + i;
+    int cell = p < end ? __ldg(rid + p) : -1;
+    const bool ok = cell >= 0 && cell < a.max_cells;
+    if (!ok) cell = 0;
+    const size_t row = (static_cast<size_t>(cell) * kHKV + kvh) * kD + part * 16;
+    cp_async16(st.k + i * kAttnKStride + part * 16, a.k + row, ok);
+    cp_async16(st.v + i * kAttnVStride + part * 16, a.v + row, ok);
+  }
+  if (tid < 2 * kAttnCells) {
+    const int i = tid & 31;
+    const int p = pos0 + i;
+    int cell = p < end ? __ldg(rid + p) : -1;
+    const bool ok = cell >= 0 && cell < a.max_cells;
+    if (tid < kAttnCells) st.valid[i] = ok;
+    if (!ok) cell = 0;
+    const size_t srow = (static_cast<size_t>(cell) * kHKV + kvh) * kNG;
+    if (tid < kAttnCells) cp_async16(st.ks + i * kNG, a.ks + srow, ok);
+    else cp_async16(st.vs + i * kNG, a.vs + srow, ok);
+  }
+}
+
+// grid: (nsplit, 2, rows); block: 128 threads; dynamic smem: sizeof(AttnSmem).
+__global__ void __launch_bounds__(128) attn_kernel(AttnArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  AttnSmem& sm = *reinterpret_cast<AttnSmem*>(smem_raw);
+  const int split = blockIdx.x, kvh = blockIdx.y, row = blockIdx.z;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int beg = min(a.top_k, split * a.piece);
+  const int end = min(a.top_k, beg + a.piece);
+  const int* rid = a.ids + static_cast<size_t>(row) * a.top_k;
+  const int nblk = (end - beg + kAttnCells - 1) / kAttnCells;
+
+  if (nblk > 0) attn_issue(sm.st[0], a, rid, beg, end, kvh);
+  cp_async_commit();
+
+  // Q fragments for this warp's two scale groups (dims [64w, 64w+64)), prescaled.
+  // Within group qg, thread t covers dims 32qg + 8t + 4s + {0..3} in sub-step s:
+  // k-index 2t,2t+1 <-> +0,+1 and 2t+8,2t+9 <-> +2,+3 (the same map as the K loads).
+  uint32_t aq[2][2][4];
+  {
+    const float* q0 = a.q + (static_cast<size_t>(row) * kHQ + kvh * kQPerKV + g) * kD;
+    const float* q8 = q0 + 8 * kD;
+    const bool has8 = g + 8 < kQPerKV;
+#pragma unroll
+    for (int gi = 0; gi < 2; ++gi)
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        const int d0 = 32 * (2 * warp + gi) + 8 * t + 4 * s;
+        const float4 x = __ldg(reinterpret_cast<const float4*>(q0 + d0));
+        const float sl = a.scale_log2;
+        aq[gi][s][0] = pack_half2(x.x * sl, x.y * sl);
+        aq[gi][s][2] = pack_half2(x.z * sl, x.w * sl);
+        if (has8) {
+          const float4 y = __ldg(reinterpret_cast<const float4*>(q8 + d0));
+          aq[gi][s][1] = pack_half2(y.x * sl, y.y * sl);
+          aq[gi][s][3] = pack_half2(y.z * sl, y.w * sl);
+        } else {
+          aq[gi][s][1] = 0u;
+          aq[gi][s][3] = 0u;
+        }
+      }
+  }
+
+  float m_run[2] = {-INFINITY, -INFINITY};
+  float l_run[2] = {0.f, 0.f};
+  float o[2][4][4];
+#pragma unroll
+  for (int gi = 0; gi < 2; ++gi)
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) o[gi][i][c] = 0.f;
+
+  for (int b = 0; b < nblk; ++b) {
+    if (b + 1 < nblk) attn_issue(sm.st[(b + 1) & 1], a, rid, beg + (b + 1) * kAttnCells, end, kvh);
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncthreads();
+    const AttnStage& st = sm.st[b & 1];
+
+    // ---- partial scores over this warp's 64 dims
+    float s[4][4];
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) s[nt][c] = 0.f;
+      const int8_t* krow = st.k + (8 * nt + g) * kAttnKStride;
+#pragma unroll
+      for (int gi = 0; gi < 2; ++gi) {
+        const int qg = 2 * warp + gi;
+        const uint2 kw = *reinterpret_cast<const uint2*>(krow + 32 * qg + 8 * t);
+        const uint32_t x0 = kw.x ^ 0x80808080u, x1 = kw.y ^ 0x80808080u;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_f16_16816(acc, aq[gi][0], i8x2_to_h2(x0, 0x4140u), i8x2_to_h2(x0, 0x4342u));
+        mma_f16_16816(acc, aq[gi][1], i8x2_to_h2(x1, 0x4140u), i8x2_to_h2(x1, 0x4342u));
+        const float sc0 = __half2float(st.ks[(8 * nt + 2 * t) * kNG + qg]);
+        const float sc1 = __half2float(st.ks[(8 * nt + 2 * t + 1) * kNG + qg]);
+        s[nt][0] = fmaf(sc0, acc[0], s[nt][0]);
+        s[nt][1] = fmaf(sc1, acc[1], s[nt][1]);
+        s[nt][2] = fmaf(sc0, acc[2], s[nt][2]);
+        s[nt][3] = fmaf(sc1, acc[3], s[nt][3]);
+      }
+      sm.red[warp][nt][lane] = make_float4(s[nt][0], s[nt][1], s[nt][2], s[nt][3]);
+    }
+    __syncthreads();
+    // ---- full scores (same summation order in every warp), masked
+    float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      float4 r = sm.red[0][nt][lane];
+#pragma unroll
+      for (int w = 1; w < 4; ++w) {
+        const float4 y = sm.red[w][nt][lane];
+        r.x += y.x;
+        r.y += y.y;
+        r.z += y.z;
+        r.w += y.w;
+      }
+      const bool v0 = st.valid[8 * nt + 2 * t], v1 = st.valid[8 * nt + 2 * t + 1];
+      s[nt][0] = v0 ? r.x : -INFINITY;
+      s[nt][1] = v1 ? r.y : -INFINITY;
+      s[nt][2] = v0 ? r.z : -INFINITY;
+      s[nt][3] = v1 ? r.w : -INFINITY;
+      mx[0] = fmaxf(mx[0], fmaxf(s[nt][0], s[nt][1]));
+      mx[1] = fmaxf(mx[1], fmaxf(s[nt][2], s[nt][3]));
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+      mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+    }
+    float alpha[2], mnew[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      mnew[r] = fmaxf(m_run[r], mx[r]);
+      alpha[r] = (mnew[r] == -INFINITY) ? 1.f : exp2f(m_run[r] - mnew[r]);
+    }
+    float rs[2] = {0.f, 0.f};
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int r = c >> 1;
+        const float p = (mnew[r] == -INFINITY) ? 0.f : exp2f(s[nt][c] - mnew[r]);
+        s[nt][c] = p;
+        rs[r] += p;
+      }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      rs[r] += __shfl_xor_sync(0xffffffffu, rs[r], 1);
+      rs[r] += __shfl_xor_sync(0xffffffffu, rs[r], 2);
+      l_run[r] = l_run[r] * alpha[r] + rs[r];
+      m_run[r] = mnew[r];
+    }
+#pragma unroll
+    for (int gi = 0; gi < 2; ++gi)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        o[gi][i][0] *= alpha[0];
+        o[gi][i][1] *= alpha[0];
+        o[gi][i][2] *= alpha[1];
+        o[gi][i][3] *= alpha[1];
+      }
+
+    // ---- P.V for this warp's 64 dims; P's k-index j <-> cell 16*s2 + j
+#pragma unroll
+    for (int s2 = 0; s2 < 2; ++s2) {
+      uint32_t pa[4];
+      pa[0] = pack_half2(s[2 * s2][0], s[2 * s2][1]);
+      pa[1] = pack_half2(s[2 * s2][2], s[2 * s2][3]);
+      pa[2] = pack_half2(s[2 * s2 + 1][0], s[2 * s2 + 1][1]);
+      pa[3] = pack_half2(s[2 * s2 + 1][2], s[2 * s2 + 1][3]);
+      const int cA = 16 * s2 + 2 * t;  // cells of k-index 2t, 2t+1, 2t+8, 2t+9
+#pragma unroll
+      for (int gi = 0; gi < 2; ++gi) {
+        const int qg = 2 * warp + gi;
+        // column g of n-tile i is dim 32qg + 4g + i
+        const int8_t* vb = st.v + 32 * qg + 4 * g;
+        const uint32_t wA = *reinterpret_cast<const uint32_t*>(vb + cA * kAttnVStride) ^ 0x80808080u;
+        const uint32_t wB = *reinterpret_cast<const uint32_t*>(vb + (cA + 1) * kAttnVStride) ^ 0x80808080u;
+        const uint32_t wC = *reinterpret_cast<const uint32_t*>(vb + (cA + 8) * kAttnVStride) ^ 0x80808080u;
+        const uint32_t wD = *reinterpret_cast<const uint32_t*>(vb + (cA + 9) * kAttnVStride) ^ 0x80808080u;
+        const __half2 sAB = __halves2half2(st.vs[cA * kNG + qg], st.vs[(cA + 1) * kNG + qg]);
+        const __half2 sCD = __halves2half2(st.vs[(cA + 8) * kNG + qg], st.vs[(cA + 9) * kNG + qg]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          uint32_t b0 = i8_pair_to_h2(wA, wB, i);
+          uint32_t b1 = i8_pair_to_h2(wC, wD, i);
+          const __half2 h0 = __hmul2(*reinterpret_cast<const __half2*>(&b0), sAB);
+          const __half2 h1 = __hmul2(*reinterpret_cast<const __half2*>(&b1), sCD);
+          mma_f16_16816(o[gi][i], pa, *reinterpret_cast<const uint32_t*>(&h0),
+                        *reinterpret_cast<const uint32_t*>(&h1));
+        }
+      }
+    }
+    __syncthreads();
+  }
+  cp_async_wait<0>();
+
+  // ---- epilogue: rows g (heads 12kvh + g) and g + 8 (heads 12kvh + g + 8, g < 4)
+  // C element (row, col 2t) of n-tile i, group qg is dim 32qg + 8t + i; col 2t+1 is +4.
+  const float kLn2 = 0.6931471805599453f;
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int hr = g + 8 * r;
+    if (hr >= kQPerKV) continue;
+    const int head = kvh * kQPerKV + hr;
+    const size_t rh = static_cast<size_t>(row) * kHQ + head;
+#pragma unroll
+    for (int gi = 0; gi < 2; ++gi) {
+      const int dbase = 32 * (2 * warp + gi) + 8 * t;
+      float4 lo = make_float4(o[gi][0][2 * r], o[gi][1][2 * r], o[gi][2][2 * r], o[gi][3][2 * r]);
+      float4 hi = make_float4(o[gi][0][2 * r + 1], o[gi][1][2 * r + 1], o[gi][2][2 * r + 1],
+                              o[gi][3][2 * r + 1]);
+      if (a.nsplit == 1) {
+        const float inv = l_run[r] > 0.f ? 1.f / l_run[r] : 0.f;
+        lo.x *= inv; lo.y *= inv; lo.z *= inv; lo.w *= inv;
+        hi.x *= inv; hi.y *= inv; hi.z *= inv; hi.w *= inv;
+        float* dst = a.out + rh * kD + dbase;
+        *reinterpret_cast<float4*>(dst) = lo;
+        *reinterpret_cast<float4*>(dst + 4) = hi;
+      } else {
+        float* dst = a.part + (rh * a.nsplit + split) * kPart;
+        *reinterpret_cast<float2*>(dst + 2 + dbase) = make_float2(lo.x, lo.y);
+        *reinterpret_cast<float2*>(dst + 2 + dbase + 2) = make_float2(lo.z, lo.w);
+        *reinterpret_cast<float2*>(dst + 2 + dbase + 4) = make_float2(hi.x, hi.y);
+        *reinterpret_cast<float2*>(dst + 2 + dbase + 6) = make_float2(hi.z, hi.w);
+        if (warp == 0 && t == 0) {
+          dst[0] = m_run[r] == -INFINITY ? -INFINITY : m_run[r] * kLn2;
+          dst[1] = l_run[r];
+        }
+      }
+    }
+  }
+}
+
+}  // namespace qsa
