@@ -23,7 +23,8 @@
  * Conventions for every call:
  *   - Pointers are CUDA device pointers owned by the caller unless stated.
  *     The library never allocates, frees or synchronises, and keeps no state
- *     between calls apart from the launch counter and the last error string.
+ *     between calls apart from the launch counter, the last error string and
+ *     the fixed scratch buffer of qsa_topk_static.
  *   - fp16 values travel as their IEEE binary16 bit patterns (uint16_t).
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream); every call
  *     only enqueues kernels on it and returns.  Results are ready when the
@@ -193,6 +194,35 @@ int qsa_attn(const qsa_cache* cache, int rows, const float* q, const int32_t* id
  * (0 when every piece is empty).  part as written by qsa_attn.
  */
 int qsa_merge(const float* part, int rows, int nsplit, float* out, void* stream);
+
+/*
+ * Selection without a caller workspace.  The pages have no counterpart to this
+ * call; it exists for callers that cannot allocate device memory when they need
+ * a selection -- code running while a CUDA graph is being captured (an
+ * allocation cannot be recorded into a graph), serving loops that must not pay
+ * for an allocator call or its implicit device synchronisation, and runtimes
+ * whose device memory is already fully owned by another allocator.
+ *
+ * It computes exactly what qsa_topk computes (same arguments, minus the
+ * workspace), using a fixed scratch buffer of QSA_STATIC_SCRATCH_BYTES that
+ * the library holds in global memory on every GPU that loads it, until the
+ * process exits.  Limits: rows <= QSA_STATIC_MAX_ROWS and
+ * top_k <= QSA_STATIC_MAX_TOPK; larger requests return QSA_ERR_ARG and
+ * launch nothing.  It never allocates or frees memory.
+ *
+ * The first call on each device looks up the buffer's device address (with
+ * that device current), so make that first call before any stream capture
+ * that is to contain later calls.  All calls on a device share the one
+ * buffer, and each call clears the parts that must start at zero: calls
+ * that can run at the same time on the GPU (different streams, or threads
+ * without ordering between them) race on it and must be serialised, for
+ * example by issuing them on one stream.
+ */
+#define QSA_STATIC_MAX_ROWS 8
+#define QSA_STATIC_MAX_TOPK 2048
+#define QSA_STATIC_SCRATCH_BYTES 1179904
+int qsa_topk_static(const float* scores, int64_t ld, int rows, int vis0, int top_k, int32_t* ids,
+                    void* stream);
 
 /* Text of the last error on the calling thread ("" when none). */
 const char* qsa_last_error(void);

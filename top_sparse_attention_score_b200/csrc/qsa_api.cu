@@ -7,6 +7,7 @@
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
+#include <mutex>
 #include <string>
 
 #include "qsa.h"
@@ -362,3 +363,66 @@ const char* qsa_last_error(void) { return g_error.c_str(); }
 uint64_t qsa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 }  // extern "C"
+
+// ---- selection without a caller workspace ----------------------------------
+//
+// A fixed scratch buffer in global memory replaces the workspace for callers
+// that cannot allocate (see qsa_topk_static in include/qsa.h).  Host code must
+// not pass the symbol itself to a kernel -- on the host it names a stand-in, not
+// device memory -- so its device address is looked up once per device.
+
+static __device__ __align__(256) unsigned char g_topk_static_scratch[QSA_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_static_mu;
+void* g_static_addr[64] = {};
+
+// Device address of the scratch buffer on the current device (looked up on first use).
+int static_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= 64) return fail(QSA_ERR_ARG, "device %d outside the 64 this library tracks", dev);
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_topk_static_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(QSA_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+    g_static_addr[dev] = p;
+  }
+  *out = g_static_addr[dev];
+  return QSA_OK;
+}
+
+}  // namespace
+
+extern "C" int qsa_topk_static(const float* scores, int64_t ld, int rows, int vis0, int top_k,
+                               int32_t* ids, void* stream) {
+  if (!scores || !ids) return fail(QSA_ERR_ARG, "scores and ids must not be NULL");
+  if (rows < 1 || rows > QSA_STATIC_MAX_ROWS)
+    return fail(QSA_ERR_ARG, "rows = %d outside [1, %d] (the fixed scratch holds %d rows)", rows,
+                QSA_STATIC_MAX_ROWS, QSA_STATIC_MAX_ROWS);
+  if (top_k < 1 || top_k > QSA_STATIC_MAX_TOPK)
+    return fail(QSA_ERR_ARG, "top_k = %d outside [1, %d] (the fixed scratch limit)", top_k,
+                QSA_STATIC_MAX_TOPK);
+  if (vis0 < 1) return fail(QSA_ERR_ARG, "vis0 = %d must be >= 1", vis0);
+  const int64_t vmax = static_cast<int64_t>(vis0) + rows - 1;
+  if (vmax > ld || ld % 4 || vmax > QSA_MAX_CELLS)
+    return fail(QSA_ERR_ARG, "rows see up to %lld cells but ld = %lld (must be >= and a multiple of 4)",
+                static_cast<long long>(vmax), static_cast<long long>(ld));
+  if (!aligned16(scores) || !aligned16(ids)) return fail(QSA_ERR_ARG, "scores and ids must be 16-byte aligned");
+  const TopkPlan p = plan_topk(0, rows, static_cast<int>(vmax), top_k);
+  if (p.end > QSA_STATIC_SCRATCH_BYTES)
+    return fail(QSA_ERR_ARG, "selection needs %zu bytes of scratch, the fixed buffer has %d", p.end,
+                QSA_STATIC_SCRATCH_BYTES);
+  void* ws = nullptr;
+  int r = static_scratch(&ws);
+  if (r) return r;
+  if ((r = prepare_device())) return r;
+  // launch_topk clears the histogram and counters before every use.
+  if ((r = launch_topk(scores, ld, rows, vis0, top_k, ws, p, ids, static_cast<cudaStream_t>(stream))))
+    return r;
+  return ok();
+}

@@ -39,6 +39,7 @@ SIGNATURES = {
     "qsa_topk": (_I, [_P, _I64, _I, _I, _I, _P, _SZ, _P, _P]),
     "qsa_attn": (_I, [_P, _I, _P, _P, _I, _I, _F, _P, _P, _P]),
     "qsa_merge": (_I, [_P, _I, _I, _P, _P]),
+    "qsa_topk_static": (_I, [_P, _I64, _I, _I, _I, _P, _P]),
     "qsa_last_error": (ctypes.c_char_p, []),
     "qsa_launch_count": (ctypes.c_uint64, []),
 }
