@@ -32,7 +32,8 @@
  *   - Return codes: QSA_OK, or QSA_ERR_ARG (bad argument: nothing launched),
  *     QSA_ERR_WORKSPACE (workspace too small: nothing launched), QSA_ERR_CUDA
  *     (a launch failed; qsa_last_error() says which).  QSA_ERR_TIMEOUT is
- *     reserved: no kernel here waits on another, so none can time out.
+ *     reported through qsa_device_status: the calls are asynchronous, so a
+ *     kernel's bounded wait that expires cannot return it directly.
  *   - Arrays must be 16-byte aligned (cudaMalloc and torch allocations are).
  *   - Non-finite inputs (NaN, inf) give unspecified results.
  */
@@ -220,9 +221,27 @@ int qsa_merge(const float* part, int rows, int nsplit, float* out, void* stream)
  */
 #define QSA_STATIC_MAX_ROWS 8
 #define QSA_STATIC_MAX_TOPK 2048
-#define QSA_STATIC_SCRATCH_BYTES 1179904
+#define QSA_STATIC_SCRATCH_BYTES 1183744
 int qsa_topk_static(const float* scores, int64_t ld, int rows, int vis0, int top_k, int32_t* ids,
                     void* stream);
+
+/*
+ * Device-side failure report.  Kernels that wait on an mbarrier (the prefill
+ * score GEMM) bound every wait to one second; on expiry they stop, drain their
+ * copies, free their tensor memory and record QSA_ERR_TIMEOUT in a status word
+ * of the current device.  This call copies that word into *status (QSA_OK or
+ * QSA_ERR_TIMEOUT) and clears it.  Unlike the other calls it synchronises
+ * `stream`.
+ */
+int qsa_device_status(int* status, void* stream);
+
+/*
+ * Self-test of that mechanism: enqueues one kernel that waits on a barrier
+ * nothing completes; after about one second it gives up and records
+ * QSA_ERR_TIMEOUT, which qsa_device_status then reports.  The context stays
+ * usable.
+ */
+int qsa_selftest_wait_timeout(void* stream);
 
 /* Text of the last error on the calling thread ("" when none). */
 const char* qsa_last_error(void);

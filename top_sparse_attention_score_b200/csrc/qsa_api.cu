@@ -1,7 +1,9 @@
 // qsa_api.cu -- the C ABI declared in include/qsa.h: argument checks, workspace
 // planning and kernel launches.  Every step of the computation runs in the
 // kernels of the qsa_*.cuh files; nothing here touches the data.
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <algorithm>
 #include <atomic>
@@ -9,6 +11,7 @@
 #include <cstdio>
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include "qsa.h"
 #include "qsa_attn.cuh"
@@ -16,7 +19,13 @@
 #include "qsa_common.cuh"
 #include "qsa_index_score.cuh"
 #include "qsa_merge.cuh"
+#include "qsa_score_gemm.cuh"
 #include "qsa_topk.cuh"
+#include "qsa_topk_cluster.cuh"
+
+// One status word per device: a kernel whose bounded wait expires records
+// QSA_ERR_TIMEOUT here (read and cleared by qsa_device_status).
+static __device__ uint32_t g_device_status;
 
 namespace {
 
@@ -46,6 +55,25 @@ int launched(const char* what) {
   return QSA_OK;
 }
 
+// Launch with programmatic stream serialisation: the kernel may be scheduled
+// while its predecessor on the stream drains; every kernel here waits on
+// griddepcontrol.wait before touching memory its predecessors use.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -62,22 +90,50 @@ int check_cache(const qsa_cache* c) {
   return QSA_OK;
 }
 
-// Opt the kernels that need it into large dynamic shared memory, once per device.
+int g_sm_count[64] = {};
+uint32_t* g_status_addr[64] = {};
+
+// Opt the kernels that need it into large dynamic shared memory and read the
+// SM count, once per device.
 int prepare_device() {
   static std::atomic<uint64_t> done_mask{0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaGetDevice failed");
   const uint64_t bit = 1ull << (dev & 63);
   if (done_mask.load() & bit) return QSA_OK;
-  cudaError_t e = cudaFuncSetAttribute(qsa::topk_final_kernel,
+  cudaError_t e = cudaFuncSetAttribute(qsa::topk_select_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        2 * (qsa::kMaxWindowBits / 32) * 4);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(qsa::attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(sizeof(qsa::AttnSmem)));
-  if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(qsa::cluster_select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             64 * qsa::kClusterThreads * 4);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(qsa::score_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             qsa::kGemmSmemRequest);
+  void* status = nullptr;
+  if (e == cudaSuccess) e = cudaGetSymbolAddress(&status, g_device_status);
+  int sms = 0;
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "device set-up: %s", cudaGetErrorString(e));
+  g_sm_count[dev & 63] = sms;
+  g_status_addr[dev & 63] = static_cast<uint32_t*>(status);
   done_mask.fetch_or(bit);
   return QSA_OK;
+}
+
+uint32_t* device_status() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return g_status_addr[dev & 63];
+}
+
+int sm_count() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return g_sm_count[dev & 63] > 0 ? g_sm_count[dev & 63] : 148;
 }
 
 // ---- workspace plan -------------------------------------------------------
@@ -92,7 +148,7 @@ TopkPlan plan_topk(size_t at, int rows, int vmax, int top_k) {
   p.cand_cap = std::min(vmax, std::max(8 * top_k, 16384));
   p.hist = align_up(at, 256);
   p.ctr = align_up(p.hist + static_cast<size_t>(rows) * qsa::kBins * 4, 256);
-  p.sure = align_up(p.ctr + static_cast<size_t>(rows) * 4 * 4, 256);
+  p.sure = align_up(p.ctr + (static_cast<size_t>(rows) * qsa::kCtrWords + 4) * 4, 256);
   p.cand = align_up(p.sure + static_cast<size_t>(rows) * top_k * 4, 256);
   p.end = align_up(p.cand + static_cast<size_t>(rows) * p.cand_cap * 8, 256);
   return p;
@@ -119,8 +175,9 @@ struct StepPlan {
 };
 
 int auto_nsplit(int rows, int top_k) {
-  // Enough (row, KV head, split) CTAs to cover the 148 SMs twice, pieces of >= 32 cells.
-  const int want = (2 * 148 + 2 * rows - 1) / (2 * rows);
+  // As many (row, KV head, split) CTAs as one wave holds (4 per SM on 148 SMs),
+  // pieces of at least 32 cells; large prefill chunks need no splits.
+  const int want = (4 * 148) / (2 * rows);
   return std::max(1, std::min({QSA_MAX_SPLITS, std::max(1, top_k / 32), want}));
 }
 
@@ -140,36 +197,154 @@ StepPlan plan_step(int rows, int ncells, int vmax, int top_k, int nsplit) {
 
 // ---- launches -------------------------------------------------------------
 
+PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
+std::mutex g_encode_mu;
+
+int tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000* out) {
+  std::lock_guard<std::mutex> lock(g_encode_mu);
+  if (!g_encode_tiled) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    const cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+      return fail(QSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+    g_encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  *out = g_encode_tiled;
+  return QSA_OK;
+}
+
+// Scores of `rows` > 8 rows: the tcgen05 GEMM, keys and queries fed by TMA.
+int launch_score_gemm(const qsa_cache* c, int rows, int ncells, const uint16_t* iq, const float* iw,
+                      float* scores, int64_t ld, cudaStream_t s) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  int r = tensor_map_encoder(&encode);
+  if (r) return r;
+  CUtensorMap tkey, tiq;
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(QSA_DI), static_cast<cuuint64_t>(ncells)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(QSA_DI) * 2};
+    const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(qsa::kGemmCells)};
+    const cuuint32_t estr[2] = {1u, 1u};
+    const CUresult cr = encode(&tkey, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->idx_key, dims, strides, box, estr,
+                               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return fail(QSA_ERR_CUDA, "tensor map of the keys: error %d", static_cast<int>(cr));
+  }
+  {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(QSA_DI), static_cast<cuuint64_t>(QSA_HI),
+                                static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(QSA_DI) * 2, static_cast<cuuint64_t>(QSA_HI * QSA_DI) * 2};
+    const cuuint32_t box[3] = {64u, 1u, static_cast<cuuint32_t>(qsa::kGemmTokens)};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    const CUresult cr = encode(&tiq, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<uint16_t*>(iq), dims, strides,
+                               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return fail(QSA_ERR_CUDA, "tensor map of the queries: error %d", static_cast<int>(cr));
+  }
+  qsa::GemmArgs a;
+  a.iw = iw;
+  a.scores = scores;
+  a.ld = ld;
+  a.T = rows;
+  a.ncells = ncells;
+  a.status = device_status();
+  const int items = ((rows + qsa::kGemmTokens - 1) / qsa::kGemmTokens) *
+                    ((ncells + qsa::kGemmCells - 1) / qsa::kGemmCells);
+  const dim3 grid(std::max(1, std::min(items, sm_count())));
+  launch_pdl(qsa::score_gemm_kernel, grid, dim3(qsa::kGemmThreads), qsa::kGemmSmemRequest, s, tkey, tiq, a);
+  return launched("score_gemm_kernel");
+}
+
 int launch_index_score(const qsa_cache* c, int rows, int ncells, const uint16_t* iq,
                        const float* iw, float* scores, int64_t ld, cudaStream_t s) {
+  if (rows > qsa::kScoreRowsPerCta) return launch_score_gemm(c, rows, ncells, iq, iw, scores, ld, s);
   const dim3 grid((ncells + qsa::kScoreCellsPerCta - 1) / qsa::kScoreCellsPerCta,
                   (rows + qsa::kScoreRowsPerCta - 1) / qsa::kScoreRowsPerCta);
-  qsa::index_score_kernel<<<grid, 128, 0, s>>>(reinterpret_cast<const __half*>(c->idx_key), ncells,
-                                               reinterpret_cast<const __half*>(iq), iw, rows,
-                                               scores, ld);
+  launch_pdl(qsa::index_score_kernel, grid, dim3(128), 0, s,
+             reinterpret_cast<const __half*>(c->idx_key), ncells, reinterpret_cast<const __half*>(iq),
+             iw, rows, scores, ld);
   return launched("index_score_kernel");
 }
 
+int launch_zero(void* ws, const TopkPlan& p, cudaStream_t s) {
+  // hist and ctr are adjacent up to alignment padding; zero both regions.
+  const int64_t nzero = static_cast<int64_t>((p.sure - p.hist) / 4);
+  const int zblocks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(592, (nzero + 255) / 256)));
+  launch_pdl(qsa::topk_zero_kernel, dim3(zblocks), dim3(256), 0, s,
+             reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + p.hist), nzero);
+  return launched("topk_zero_kernel");
+}
+
+int launch_select(const float* scores, int64_t ld, int rows, int vis0, int top_k,
+                  const qsa::TopkWs& w, int32_t* ids, cudaStream_t s) {
+  const int vmax = vis0 + rows - 1;
+  const dim3 grid((vmax + qsa::kTopkChunk - 1) / qsa::kTopkChunk, rows);
+  const int win = std::min(qsa::kMaxWindowBits, static_cast<int>(align_up(vmax, 32)));
+  const size_t smem = 2 * static_cast<size_t>(win / 32) * 4;
+  launch_pdl(qsa::topk_select_kernel, grid, dim3(qsa::kTopkThreads), smem, s, scores, ld, vis0, top_k,
+             w, win, ids);
+  return launched("topk_select_kernel");
+}
+
+// Selection over given scores: zero, histogram (+ thresholds), select.
 int launch_topk(const float* scores, int64_t ld, int rows, int vis0, int top_k, void* ws,
                 const TopkPlan& p, int32_t* ids, cudaStream_t s) {
   const qsa::TopkWs w = topk_ws(ws, p);
   const int vmax = vis0 + rows - 1;
-  // hist and ctr are adjacent up to alignment padding; zero both regions.
-  const int64_t nzero = static_cast<int64_t>((p.sure - p.hist) / 4);
-  const int zblocks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(592, (nzero + 255) / 256)));
-  qsa::topk_zero_kernel<<<zblocks, 256, 0, s>>>(w.hist, nzero);
-  int r = launched("topk_zero_kernel");
+  int r = launch_zero(ws, p, s);
   if (r) return r;
   const dim3 grid((vmax + qsa::kTopkChunk - 1) / qsa::kTopkChunk, rows);
-  qsa::topk_hist_kernel<<<grid, qsa::kTopkThreads, 0, s>>>(scores, ld, vis0, top_k, w);
+  launch_pdl(qsa::topk_hist_kernel, grid, dim3(qsa::kTopkThreads), 0, s, scores, ld, vis0, top_k, w);
   if ((r = launched("topk_hist_kernel"))) return r;
-  qsa::topk_filter_kernel<<<grid, qsa::kTopkThreads, 0, s>>>(scores, ld, vis0, top_k, w);
-  if ((r = launched("topk_filter_kernel"))) return r;
-  const int win = std::min(qsa::kMaxWindowBits, static_cast<int>(align_up(vmax, 32)));
-  const size_t smem = 2 * static_cast<size_t>(win / 32) * 4;
-  qsa::topk_final_kernel<<<rows, qsa::kFinalThreads, smem, s>>>(scores, ld, vis0, top_k, w, win,
-                                                                ids);
-  return launched("topk_final_kernel");
+  return launch_select(scores, ld, rows, vis0, top_k, w, ids, s);
+}
+
+// Selection by one 8-CTA cluster per row (rows of at most 8 x 512 x 64 cells).
+template <int PER>
+int launch_cluster_select_per(const float* scores, int64_t ld, int rows, int vis0, int top_k,
+                              int32_t* ids, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(qsa::kClusterCtas, rows);
+  cfg.blockDim = dim3(qsa::kClusterThreads);
+  cfg.dynamicSmemBytes = PER > qsa::kClusterRegPer ? static_cast<size_t>(PER) * qsa::kClusterThreads * 4 : 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = qsa::kClusterCtas;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  cudaLaunchKernelEx(&cfg, qsa::cluster_select_kernel<PER>, scores, ld, vis0, top_k, ids);
+  return launched("cluster_select_kernel");
+}
+
+constexpr int kClusterMaxCells = qsa::kClusterCtas * qsa::kClusterThreads * 64;
+
+int launch_cluster_select(const float* scores, int64_t ld, int rows, int vis0, int top_k,
+                          int32_t* ids, cudaStream_t s) {
+  const int vmax = vis0 + rows - 1;
+  const int per_cta = qsa::kClusterCtas * qsa::kClusterThreads;
+  const int need = (vmax + per_cta - 1) / per_cta;
+  if (need <= 1) return launch_cluster_select_per<1>(scores, ld, rows, vis0, top_k, ids, s);
+  if (need <= 2) return launch_cluster_select_per<2>(scores, ld, rows, vis0, top_k, ids, s);
+  if (need <= 4) return launch_cluster_select_per<4>(scores, ld, rows, vis0, top_k, ids, s);
+  if (need <= 8) return launch_cluster_select_per<8>(scores, ld, rows, vis0, top_k, ids, s);
+  if (need <= 16) return launch_cluster_select_per<16>(scores, ld, rows, vis0, top_k, ids, s);
+  if (need <= 32) return launch_cluster_select_per<32>(scores, ld, rows, vis0, top_k, ids, s);
+  return launch_cluster_select_per<64>(scores, ld, rows, vis0, top_k, ids, s);
+}
+
+// The selection used by qsa_topk and the whole-step calls: one cluster per row
+// when the rows fit one, else the multi-kernel path through the workspace.
+int launch_selection(const float* scores, int64_t ld, int rows, int vis0, int top_k, void* ws,
+                     const TopkPlan& p, int32_t* ids, cudaStream_t s) {
+  if (vis0 + rows - 1 <= kClusterMaxCells)
+    return launch_cluster_select(scores, ld, rows, vis0, top_k, ids, s);
+  return launch_topk(scores, ld, rows, vis0, top_k, ws, p, ids, s);
 }
 
 int launch_attn(const qsa_cache* c, int rows, const float* q, const int32_t* ids, int top_k,
@@ -188,13 +363,12 @@ int launch_attn(const qsa_cache* c, int rows, const float* q, const int32_t* ids
   a.scale_log2 = scale * 1.4426950408889634f;
   a.part = part;
   a.out = out;
-  const dim3 grid(nsplit, QSA_HKV, rows);
-  qsa::attn_kernel<<<grid, 128, sizeof(qsa::AttnSmem), s>>>(a);
+  launch_pdl(qsa::attn_kernel, dim3(nsplit, QSA_HKV, rows), dim3(128), sizeof(qsa::AttnSmem), s, a);
   return launched("attn_kernel");
 }
 
 int launch_merge(const float* part, int rows, int nsplit, float* out, cudaStream_t s) {
-  qsa::merge_kernel<<<rows * QSA_HQ, 256, 0, s>>>(part, nsplit, out);
+  launch_pdl(qsa::merge_kernel, dim3(rows * QSA_HQ), dim3(256), 0, s, part, nsplit, out);
   return launched("merge_kernel");
 }
 
@@ -218,7 +392,7 @@ int run_step(const qsa_cache* c, int rows, int vis0, int ncells, const float* q,
   int32_t* ids = ids_out ? ids_out : reinterpret_cast<int32_t*>(base + p.ids);
   float* part = reinterpret_cast<float*>(base + p.part);
   if ((r = launch_index_score(c, rows, ncells, iq, iw, scores, p.ld, s))) return r;
-  if ((r = launch_topk(scores, p.ld, rows, vis0, top_k, base, p.topk, ids, s))) return r;
+  if ((r = launch_selection(scores, p.ld, rows, vis0, top_k, base, p.topk, ids, s))) return r;
   if ((r = launch_attn(c, rows, q, ids, top_k, nsplit, scale, part, out, s))) return r;
   if (nsplit > 1 && (r = launch_merge(part, rows, nsplit, out, s))) return r;
   return ok();
@@ -252,10 +426,10 @@ int qsa_cache_write(const qsa_cache* cache, int pos0, int n, const float* k, con
   if (n < 1 || pos0 < 0 || static_cast<int64_t>(pos0) + n > cache->max_cells)
     return fail(QSA_ERR_ARG, "cells [%d, %d + %d) outside the cache of %d", pos0, pos0, n,
                 cache->max_cells);
-  const dim3 grid(n, QSA_HKV, 2);
-  qsa::cache_write_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      cache->k, cache->v, reinterpret_cast<__half*>(cache->ks), reinterpret_cast<__half*>(cache->vs),
-      reinterpret_cast<__half*>(cache->idx_key), pos0, k, v, reinterpret_cast<const __half*>(idx_key));
+  launch_pdl(qsa::cache_write_kernel, dim3(n, QSA_HKV, 2), dim3(256), 0, static_cast<cudaStream_t>(stream),
+             cache->k, cache->v, reinterpret_cast<__half*>(cache->ks), reinterpret_cast<__half*>(cache->vs),
+             reinterpret_cast<__half*>(cache->idx_key), pos0, k, v,
+             reinterpret_cast<const __half*>(idx_key));
   if ((r = launched("cache_write_kernel"))) return r;
   return ok();
 }
@@ -299,6 +473,7 @@ int qsa_index_score(const qsa_cache* cache, int rows, int ncells, const uint16_t
   if (ld < ncells || ld % 4) return fail(QSA_ERR_ARG, "ld = %lld must be >= ncells and a multiple of 4",
                                          static_cast<long long>(ld));
   if (!aligned16(iq) || !aligned16(scores)) return fail(QSA_ERR_ARG, "iq and scores must be 16-byte aligned");
+  if ((r = prepare_device())) return r;
   if ((r = launch_index_score(cache, rows, ncells, iq, iw, scores, ld,
                               static_cast<cudaStream_t>(stream))))
     return r;
@@ -326,7 +501,7 @@ int qsa_topk(const float* scores, int64_t ld, int rows, int vis0, int top_k, voi
   if (!aligned16(ws)) return fail(QSA_ERR_ARG, "ws must be 16-byte aligned");
   int r = prepare_device();
   if (r) return r;
-  if ((r = launch_topk(scores, ld, rows, vis0, top_k, ws, p, ids, static_cast<cudaStream_t>(stream))))
+  if ((r = launch_selection(scores, ld, rows, vis0, top_k, ws, p, ids, static_cast<cudaStream_t>(stream))))
     return r;
   return ok();
 }
@@ -355,6 +530,30 @@ int qsa_merge(const float* part, int rows, int nsplit, float* out, void* stream)
     return fail(QSA_ERR_ARG, "rows = %d, nsplit = %d out of range", rows, nsplit);
   int r = launch_merge(part, rows, nsplit, out, static_cast<cudaStream_t>(stream));
   if (r) return r;
+  return ok();
+}
+
+int qsa_device_status(int* status, void* stream) {
+  if (!status) return fail(QSA_ERR_ARG, "status must not be NULL");
+  int r = prepare_device();
+  if (r) return r;
+  uint32_t* addr = device_status();
+  uint32_t host = 0u;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(&host, addr, sizeof(host), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(addr, 0, sizeof(uint32_t), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "reading the device status: %s", cudaGetErrorString(e));
+  *status = static_cast<int>(host);
+  return ok();
+}
+
+int qsa_selftest_wait_timeout(void* stream) {
+  int r = prepare_device();
+  if (r) return r;
+  qsa::wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(device_status());
+  if ((r = launched("wait_selftest_kernel"))) return r;
   return ok();
 }
 

@@ -9,7 +9,7 @@
 //    tensor cores instead of 6144 fp32 FMAs per gathered cell;
 //  * cells are gathered 32 at a time with cp.async (16-byte copies of whole
 //    256-byte K/V rows and their scales) into a double-buffered shared-memory
-//    stage, so the next block's gathers are in flight while this one computes;
+//    ring, so the next block's gathers are in flight while one computes;
 //  * the four warps split the 256 dims: each computes a partial QK^T over its
 //    64 dims (two scale groups), the partials are summed through shared memory
 //    in a fixed order (all warps get bit-equal scores), each warp runs the same
@@ -35,8 +35,10 @@ struct __align__(16) AttnStage {
   int valid[kAttnCells];
 };
 
+constexpr int kAttnStages = 2;
+
 struct AttnSmem {
-  AttnStage st[2];
+  AttnStage st[kAttnStages];
   float4 red[4][4][32];  // [warp][n-tile][lane] partial scores
 };
 
@@ -96,9 +98,7 @@ __global__ void __launch_bounds__(128) attn_kernel(AttnArgs a) {
   const int end = min(a.top_k, beg + a.piece);
   const int* rid = a.ids + static_cast<size_t>(row) * a.top_k;
   const int nblk = (end - beg + kAttnCells - 1) / kAttnCells;
-
-  if (nblk > 0) attn_issue(sm.st[0], a, rid, beg, end, kvh);
-  cp_async_commit();
+  griddep_launch();
 
   // Q fragments for this warp's two scale groups (dims [64w, 64w+64)), prescaled.
   // Within group qg, thread t covers dims 32qg + 8t + 4s + {0..3} in sub-step s:
@@ -128,6 +128,14 @@ __global__ void __launch_bounds__(128) attn_kernel(AttnArgs a) {
       }
   }
 
+  // The ids come from the selection kernel: wait for it before the first gather.
+  griddep_wait();
+#pragma unroll
+  for (int st = 0; st < kAttnStages - 1; ++st) {
+    if (st < nblk) attn_issue(sm.st[st], a, rid, beg + st * kAttnCells, end, kvh);
+    cp_async_commit();
+  }
+
   float m_run[2] = {-INFINITY, -INFINITY};
   float l_run[2] = {0.f, 0.f};
   float o[2][4][4];
@@ -139,11 +147,13 @@ __global__ void __launch_bounds__(128) attn_kernel(AttnArgs a) {
       for (int c = 0; c < 4; ++c) o[gi][i][c] = 0.f;
 
   for (int b = 0; b < nblk; ++b) {
-    if (b + 1 < nblk) attn_issue(sm.st[(b + 1) & 1], a, rid, beg + (b + 1) * kAttnCells, end, kvh);
+    // refill the stage block b - 1 used (every warp finished it at the last barrier)
+    const int nb = b + kAttnStages - 1;
+    if (nb < nblk) attn_issue(sm.st[nb % kAttnStages], a, rid, beg + nb * kAttnCells, end, kvh);
     cp_async_commit();
-    cp_async_wait<1>();
+    cp_async_wait<kAttnStages - 1>();
     __syncthreads();
-    const AttnStage& st = sm.st[b & 1];
+    const AttnStage& st = sm.st[b % kAttnStages];
 
     // ---- partial scores over this warp's 64 dims
     float s[4][4];

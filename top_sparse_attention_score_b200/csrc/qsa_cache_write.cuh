@@ -22,6 +22,8 @@ __global__ void __launch_bounds__(256) cache_write_kernel(int8_t* __restrict__ k
   const int i = blockIdx.x, g = blockIdx.y, which = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, grp = tid >> 5;
   const size_t cell = static_cast<size_t>(pos0) + i;
+  griddep_launch();
+  griddep_wait();  // earlier kernels on the stream may still read the cells rewritten here
   const float x = __ldg((which ? v : k) + (static_cast<size_t>(i) * kHKV + g) * kD + tid);
   float amax = fabsf(x);
 #pragma unroll

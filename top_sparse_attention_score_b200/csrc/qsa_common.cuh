@@ -140,6 +140,15 @@ __device__ __forceinline__ void find_threshold_bin(const uint32_t* hist, int nbi
   __syncthreads();
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start while its predecessor drains.  It must call
+// griddep_wait() before touching memory the predecessor reads or writes, and
+// every CTA must call it before exiting (the ordering is transitive only if
+// no kernel completes ahead of its predecessor); griddep_launch() lets its own
+// dependent start launching early.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::); }
+
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid) {
   const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
   const int n = valid ? 16 : 0;

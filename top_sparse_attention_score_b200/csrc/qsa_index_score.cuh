@@ -31,6 +31,8 @@ __global__ void __launch_bounds__(128) index_score_kernel(const __half* __restri
   const int g = lane >> 2, t = lane & 3;
   const int cb = blockIdx.x * kScoreCellsPerCta + warp * kScoreCellsPerWarp;
   const int rb = blockIdx.y * kScoreRowsPerCta;
+  griddep_launch();
+  griddep_wait();  // keys may have just been written, scores may still be read by earlier kernels
   if (cb >= ncells) return;
 
   // K index <-> dim mapping (the contraction may permute dims as long as A and
@@ -71,6 +73,7 @@ __global__ void __launch_bounds__(128) index_score_kernel(const __half* __restri
 
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
+    if (rb + 2 * j >= rows) break;  // warp-uniform: n-tile j holds rows rb+2j, rb+2j+1
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) mma_f16_16816(acc, a[ks], b[j][ks][0], b[j][ks][1]);

@@ -18,9 +18,15 @@ __global__ void __launch_bounds__(256) merge_kernel(const float* __restrict__ pa
   __shared__ float sL;
   const int tid = threadIdx.x;
   const float* base = part + static_cast<size_t>(blockIdx.x) * nsplit * kPart;
+  griddep_launch();
+  griddep_wait();  // the partials come from the attention kernel
+  // every o_j of this dim in flight at once (nsplit <= 64)
+  float ov[64];
+#pragma unroll
+  for (int j = 0; j < 64; ++j) ov[j] = j < nsplit ? __ldcg(base + j * kPart + 2 + tid) : 0.f;
   if (tid < nsplit) {
-    sm[tid] = base[tid * kPart + 0];
-    sl[tid] = base[tid * kPart + 1];
+    sm[tid] = __ldcg(base + tid * kPart + 0);
+    sl[tid] = __ldcg(base + tid * kPart + 1);
   }
   __syncthreads();
   float M = -INFINITY;
@@ -34,7 +40,9 @@ __global__ void __launch_bounds__(256) merge_kernel(const float* __restrict__ pa
     sL = L;
   }
   float o = 0.f;
-  for (int j = 0; j < nsplit; ++j) o = fmaf(base[j * kPart + 2 + tid], se[j], o);
+#pragma unroll
+  for (int j = 0; j < 64; ++j)
+    if (j < nsplit) o = fmaf(ov[j], se[j], o);
   __syncthreads();
   out[static_cast<size_t>(blockIdx.x) * kD + tid] = sL > 0.f ? o / sL : 0.f;
 }

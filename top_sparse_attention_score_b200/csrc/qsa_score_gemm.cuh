@@ -1,0 +1,378 @@
+// qsa_score_gemm.cuh -- prefill indexer scores as a tcgen05 / TMEM GEMM fed by TMA.
+//
+// The prompt path's qsa_score_mm ("opus r15 track A: prompt_chunk wave zipping, ...",
+// what changed, item 1): for T query tokens and L cells,
+//   score[t][c] = sum_h w[t][h] * max(0, sum_d iq[t][h][d] * key[c][d])   (4 heads x 64, fp16)
+// is four [T x 64] x [64 x L] products followed by a ReLU-weighted sum over heads.
+//
+// sm_100a design (one persistent CTA per SM, 10 warps):
+//   * a tile is 128 tokens x 64 cells.  For each head h one tcgen05.mma chain
+//     (M = 128, N = 64, four K = 16 steps) writes D_h = iq_h . key^T into its own
+//     64 TMEM columns, so token t's four head products sit in TMEM lane t at the
+//     same column: the epilogue combines them without any data exchange;
+//   * the 128 tokens' queries (4 heads x 128 x 64 fp16 = 64 KB) stay in shared
+//     memory while a CTA sweeps its cells; key tiles (64 x 64 fp16 = 8 KB) stream
+//     in through a 4-stage TMA ring, both with the 128-byte swizzle the UMMA
+//     K-major descriptors describe;
+//   * warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs (one thread),
+//     warps 2..9 are the epilogue.  TMEM holds two 256-column accumulators, so
+//     the epilogue of tile i overlaps the MMAs of tile i + 1;
+//   * every wait on an mbarrier is bounded (one second of %globaltimer): on
+//     expiry the CTA records QSA_ERR_TIMEOUT in `status`, every role stops,
+//     in-flight copies and MMAs are drained (again with a bound) and TMEM is freed.
+#pragma once
+
+#include <cuda.h>
+
+#include "qsa_common.cuh"
+
+namespace qsa {
+
+constexpr int kGemmTokens = 128;     // M
+constexpr int kGemmCells = 64;       // N per head
+constexpr int kGemmStages = 4;       // key-tile ring
+constexpr int kGemmEpiWarps = 8;
+constexpr int kGemmThreads = (2 + kGemmEpiWarps) * 32;
+constexpr int kGemmABytes = kHI * kGemmTokens * kDI * 2;   // 64 KB
+constexpr int kGemmBBytes = kGemmCells * kDI * 2;           // 8 KB
+constexpr int kGemmSmemBytes = kGemmABytes + kGemmStages * kGemmBBytes + 1024 /*barriers*/ + 1024 /*align*/;
+// Ask for more shared memory than two CTAs could share, so one CTA owns an SM
+// and its TMEM (the CTA allocates all 512 columns).
+constexpr int kGemmSmemRequest = 120 * 1024;
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // one second
+constexpr uint32_t kStatusTimeout = 4;                       // QSA_ERR_TIMEOUT
+
+struct GemmArgs {
+  const float* iw;     // [T][4]
+  float* scores;       // [T][ld]
+  int64_t ld;
+  int T;
+  int ncells;
+  uint32_t* status;    // 0, or QSA_ERR_TIMEOUT after a wait expired
+};
+
+struct __align__(8) GemmBarriers {
+  uint64_t b_full[kGemmStages];
+  uint64_t b_empty[kGemmStages];
+  uint64_t a_full;
+  uint64_t a_empty;
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  uint32_t abort;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
+  return t;
+}
+
+// Wait for the phase of `bar` with parity `parity`.  Returns false if the CTA
+// is aborting or the wait exceeded its limit (which starts the abort).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, GemmBarriers& gb,
+                                          uint32_t* status) {
+  const uint32_t addr = smem_u32(bar);
+  unsigned long long t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if (*reinterpret_cast<volatile uint32_t*>(&gb.abort)) return false;
+    if ((it & 255u) == 0u) {
+      const unsigned long long now = global_ns();
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > kWaitLimitNs) {
+        atomicExch(status, kStatusTimeout);
+        *reinterpret_cast<volatile uint32_t*>(&gb.abort) = 1u;
+        return false;
+      }
+    }
+  }
+}
+
+// Wait with a bound but never start an abort (used while draining).
+__device__ __forceinline__ void mbar_drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint32_t addr = smem_u32(bar);
+  const unsigned long long t0 = global_ns();
+  for (;;) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    if (done || global_ns() - t0 > kWaitLimitNs) return;
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// UMMA shared-memory descriptor: K-major operand rows of 128 bytes with the
+// 128-byte swizzle (8-row atoms of 1024 bytes: leading offset 16 B, stride 1024 B).
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (1ull << 16) | (64ull << 32) | (1ull << 46) |
+         (2ull << 61);
+}
+
+// Instruction descriptor: fp32 accumulate, fp16 A and B, both K-major, M = 128, N = 64.
+constexpr uint32_t kGemmIdesc = (1u << 4) | (static_cast<uint32_t>(kGemmCells >> 3) << 17) |
+                                (static_cast<uint32_t>(kGemmTokens >> 4) << 24);
+
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(kGemmIdesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
+
+// grid: number of SMs (persistent); block: kGemmThreads; dynamic smem: kGemmSmemRequest.
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    score_gemm_kernel(const __grid_constant__ CUtensorMap tmap_key,
+                      const __grid_constant__ CUtensorMap tmap_iq, GemmArgs a) {
+  extern __shared__ __align__(1024) unsigned char gsm_raw[];
+  unsigned char* gsm = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  unsigned char* sA = gsm;                                   // 4 heads x 16 KB
+  unsigned char* sB = gsm + kGemmABytes;                     // stages x 8 KB
+  GemmBarriers& gb = *reinterpret_cast<GemmBarriers*>(sB + kGemmStages * kGemmBBytes);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntb = (a.T + kGemmTokens - 1) / kGemmTokens;
+  const int nct = (a.ncells + kGemmCells - 1) / kGemmCells;
+  const int items = ntb * nct;
+  const int per = (items + gridDim.x - 1) / gridDim.x;
+  const int it0 = min(items, static_cast<int>(blockIdx.x) * per);
+  const int it1 = min(items, it0 + per);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kGemmStages; ++s) {
+      mbar_init(&gb.b_full[s], 1);
+      mbar_init(&gb.b_empty[s], 1);
+    }
+    mbar_init(&gb.a_full, 1);
+    mbar_init(&gb.a_empty, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&gb.acc_full[b], 1);
+      mbar_init(&gb.acc_empty[b], kGemmEpiWarps);
+    }
+    mbar_init(&gb.drain, 1);
+    gb.abort = 0u;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  if (warp == 1) {  // allocate all 512 TMEM columns (two accumulators of 4 heads x 64)
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(&gb.tmem_base)),
+                 "r"(512u));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = gb.tmem_base;
+  griddep_launch();
+  griddep_wait();  // keys and queries may come from kernels before this one
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      int cur_tb = -1, a_loads = 0, issued = 0;
+      bool ok = true;
+      for (int it = it0; it < it1 && ok; ++it) {
+        const int tb = it / nct, ct = it % nct;
+        if (tb != cur_tb) {
+          if (a_loads > 0) ok = mbar_wait(&gb.a_empty, (a_loads - 1) & 1, gb, a.status);
+          if (!ok) break;
+          mbar_expect_tx(&gb.a_full, kGemmABytes);
+          for (int h = 0; h < kHI; ++h)
+            tma_load_3d(sA + h * (kGemmTokens * kDI * 2), &tmap_iq, 0, h, tb * kGemmTokens, &gb.a_full);
+          cur_tb = tb;
+          ++a_loads;
+        }
+        const int li = it - it0, s = li % kGemmStages, round = li / kGemmStages;
+        ok = mbar_wait(&gb.b_empty[s], (round & 1) ^ 1, gb, a.status);
+        if (!ok) break;
+        mbar_expect_tx(&gb.b_full[s], kGemmBBytes);
+        tma_load_2d(sB + s * kGemmBBytes, &tmap_key, 0, ct * kGemmCells, &gb.b_full[s]);
+        issued = li + 1;
+      }
+      if (!ok) {  // drain copies still in flight before the CTA leaves
+        for (int li = max(0, issued - kGemmStages); li < issued; ++li)
+          mbar_drain_wait(&gb.b_full[li % kGemmStages], (li / kGemmStages) & 1);
+        if (a_loads > 0) mbar_drain_wait(&gb.a_full, (a_loads - 1) & 1);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      int cur_tb = -1, a_loads = 0;
+      bool ok = true;
+      for (int it = it0; it < it1 && ok; ++it) {
+        const int tb = it / nct;
+        const int li = it - it0, s = li % kGemmStages, round = li / kGemmStages;
+        const int buf = li & 1, bround = li >> 1;
+        if (tb != cur_tb) {
+          ok = mbar_wait(&gb.a_full, a_loads & 1, gb, a.status);
+          if (!ok) break;
+          cur_tb = tb;
+          ++a_loads;
+        }
+        ok = mbar_wait(&gb.b_full[s], round & 1, gb, a.status) &&
+             mbar_wait(&gb.acc_empty[buf], (bround & 1) ^ 1, gb, a.status);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t b0 = smem_u32(sB + s * kGemmBBytes);
+#pragma unroll
+        for (int h = 0; h < kHI; ++h) {
+          const uint32_t a0 = smem_u32(sA + h * (kGemmTokens * kDI * 2));
+          const uint32_t d = tmem + static_cast<uint32_t>(buf * 256 + h * kGemmCells);
+#pragma unroll
+          for (int ks = 0; ks < kDI / 16; ++ks)
+            umma_f16(d, umma_desc_sw128(a0 + ks * 32), umma_desc_sw128(b0 + ks * 32), ks > 0 ? 1u : 0u);
+        }
+        umma_commit(&gb.b_empty[s]);       // the key stage is free once these MMAs finish
+        umma_commit(&gb.acc_full[buf]);    // the accumulator is ready for the epilogue
+        const bool last_of_tb = (it + 1 == it1) || ((it + 1) / nct != tb);
+        if (last_of_tb) umma_commit(&gb.a_empty);
+      }
+      // every MMA this thread issued has completed once `drain` fires
+      umma_commit(&gb.drain);
+      mbar_drain_wait(&gb.drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue: 8 warps; warp w reads TMEM lanes 32 * (w % 4) ...
+    const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;  // columns [32 * half, 32 * half + 32) of each head
+    int cur_tb = -1;
+    float w[kHI] = {0.f, 0.f, 0.f, 0.f};
+    for (int it = it0; it < it1; ++it) {
+      const int tb = it / nct, ct = it % nct;
+      const int li = it - it0, buf = li & 1, bround = li >> 1;
+      const int row = tb * kGemmTokens + quad * 32 + lane;
+      if (tb != cur_tb) {
+#pragma unroll
+        for (int h = 0; h < kHI; ++h) w[h] = row < a.T ? __ldg(a.iw + row * kHI + h) : 0.f;
+        cur_tb = tb;
+      }
+      // one lane waits, the warp follows it (the TMEM loads below are warp-collective)
+      uint32_t ok = 1u;
+      if (lane == 0) ok = mbar_wait(&gb.acc_full[buf], bround & 1, gb, a.status) ? 1u : 0u;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      __syncwarp();
+      tc_fence_after();
+      if (!ok) break;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int col = half * 32 + q * 16;
+        uint32_t r[kHI][16];
+#pragma unroll
+        for (int h = 0; h < kHI; ++h)
+          tmem_ld16(tmem + (static_cast<uint32_t>(quad * 32) << 16) +
+                        static_cast<uint32_t>(buf * 256 + h * kGemmCells + col),
+                    r[h]);
+        tmem_ld_wait();
+        float sc[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          float sacc = w[0] * fmaxf(__uint_as_float(r[0][j]), 0.f);
+          sacc = fmaf(w[1], fmaxf(__uint_as_float(r[1][j]), 0.f), sacc);
+          sacc = fmaf(w[2], fmaxf(__uint_as_float(r[2][j]), 0.f), sacc);
+          sc[j] = fmaf(w[3], fmaxf(__uint_as_float(r[3][j]), 0.f), sacc);
+        }
+        const int c = ct * kGemmCells + col;
+        if (row < a.T) {
+          float* dst = a.scores + row * a.ld + c;
+          if (c + 16 <= a.ncells) {
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              *reinterpret_cast<float4*>(dst + 4 * v4) =
+                  make_float4(sc[4 * v4], sc[4 * v4 + 1], sc[4 * v4 + 2], sc[4 * v4 + 3]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (c + j < a.ncells) dst[j] = sc[j];
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&gb.acc_empty[buf]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(512u));
+}
+
+// Self-test of the bounded wait: one thread waits on a barrier that nothing
+// completes and must give up after the limit, recording the timeout.
+__global__ void wait_selftest_kernel(uint32_t* status) {
+  __shared__ GemmBarriers gb;
+  if (threadIdx.x == 0) {
+    mbar_init(&gb.drain, 1);
+    gb.abort = 0u;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    mbar_wait(&gb.drain, 0, gb, status);
+  }
+}
+
+}  // namespace qsa

@@ -4,42 +4,79 @@
 // prompt_chunk wave zipping, ...", what changed, item 1), one id set per token
 // (the qids row of "Round 5 Track C Report ...", section 1, Target 2).
 //
-// Radix select in three launches, so every row spreads over many SMs:
-//   hist   (many CTAs per row) 2048-bin histogram of each score's coarse bin
-//          (top 11 bits of its fp16 key) in shared memory, flushed with atomics;
-//   filter (many CTAs per row) each CTA finds the bin holding the k-th score,
-//          appends cells of higher bins to the row's "sure" list and cells of
-//          that bin, with their full 32-bit keys, to the "candidate" list
-//          (warp-aggregated atomics);
-//   final  (one CTA per row) radix-selects the exact 32-bit threshold key
-//          among the candidates (four 8-bit passes with shared histograms),
-//          takes the lowest-index cells among equal keys, and emits the ids in
-//          ascending order by compacting a bitmap of the row's cells.
-// A candidate list that overflows its capacity is not lost: the final pass
-// then re-reads the score row itself for that bin.
+// Radix select spread over many SMs, with no CTA ever waiting on another:
+//   histogram  2048-bin count of each score's coarse bin (top 11 bits of the
+//              order-preserving key of its fp16 rounding), accumulated in shared
+//              memory and flushed with atomics -- either fused into the decode
+//              score kernel or by topk_hist_kernel.  The CTA that finishes last
+//              (a fence and a counter, no waiting) finds each row's threshold bin.
+//   select     topk_select_kernel: each CTA appends the cells of its chunk above
+//              the threshold bin to the row's "sure" list and the cells in it, with
+//              their full 32-bit keys, to the "candidate" list.  The CTA of the row
+//              that finishes last then radix-selects the exact 32-bit threshold key
+//              among the candidates (four 8-bit passes), keeps the lowest-index
+//              cells among equal keys, and writes the ids in ascending order by
+//              compacting a bitmap of the row's cells.
+// A candidate list that overflows its capacity is not lost: the last CTA then
+// re-reads the score row itself for that bin.
 #pragma once
 
 #include "qsa_common.cuh"
 
 namespace qsa {
 
-constexpr int kTopkChunk = 4096;   // scores per hist/filter CTA
-constexpr int kTopkThreads = 256;  // hist/filter block
-constexpr int kFinalThreads = 1024;
-constexpr int kMaxWindowBits = 1 << 19;  // cells per bitmap window (two 64 KB bitmaps)
+constexpr int kTopkChunk = 4096;    // scores per hist/select CTA
+constexpr int kTopkThreads = 256;   // hist/select block
+constexpr int kMaxWindowBits = 1 << 18;  // cells per bitmap window (two 32 KB bitmaps)
+
+// Per-row counters, zeroed before every use.
+enum : int {
+  kCtrSure = 0, kCtrCand = 1, kCtrHistDone = 2, kCtrSelectDone = 3, kCtrThrBin = 4,
+  kCtrAbove = 5, kCtrAttnDone = 6,  // + KV head (6, 7)
+  kCtrWords = 8
+};
 
 struct TopkWs {
   uint32_t* hist;   // [rows][kBins]
-  uint32_t* ctr;    // [rows][4]: n_sure, n_cand
+  uint32_t* ctr;    // [rows][kCtrWords], then one grid-wide counter
   int32_t* sure;    // [rows][top_k]
   uint2* cand;      // [rows][cand_cap] (key, cell)
   int cand_cap;
 };
 
 __global__ void topk_zero_kernel(uint32_t* p, int64_t n) {
+  griddep_launch();
+  griddep_wait();
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x)
     p[i] = 0u;
+}
+
+// Threshold bin of one row from its global histogram (copied to shared memory
+// through L2 first: other CTAs wrote it).  Writes ctr[kCtrThrBin], ctr[kCtrAbove].
+template <int NT>
+__device__ void row_threshold(const uint32_t* ghist, uint32_t* ctr, uint32_t k, uint32_t* sh,
+                              uint32_t* scratch, uint32_t* result) {
+  for (int i = threadIdx.x; i < kBins; i += NT) sh[i] = __ldcg(ghist + i);
+  __syncthreads();
+  uint32_t thr, above;
+  find_threshold_bin<NT>(sh, kBins, k, scratch, result, thr, above);
+  if (threadIdx.x == 0) {
+    ctr[kCtrThrBin] = thr;
+    ctr[kCtrAbove] = above;
+  }
+  __syncthreads();
+}
+
+// True in every thread of the CTA that arrives last at `counter` (of `total`).
+__device__ __forceinline__ bool last_to_arrive(uint32_t* counter, uint32_t total, uint32_t* flag) {
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) *flag = (atomicAdd(counter, 1u) == total - 1u) ? 1u : 0u;
+  __syncthreads();
+  const bool last = *flag != 0u;
+  if (last) __threadfence();
+  return last;
 }
 
 // grid: x = chunks, y = rows
@@ -47,34 +84,44 @@ __global__ void __launch_bounds__(kTopkThreads) topk_hist_kernel(const float* __
                                                                  int64_t ld, int vis0, int top_k,
                                                                  TopkWs ws) {
   __shared__ uint32_t h[kBins];
+  __shared__ uint32_t scratch[33];
+  __shared__ uint32_t result[2];
+  __shared__ uint32_t flag;
+  griddep_launch();
+  // Wait before anything else, even in CTAs with no work: a kernel that finished
+  // without waiting would let its dependents overtake the kernels before it.
+  griddep_wait();
   const int row = blockIdx.y;
   const int V = vis0 + row;
-  if (V <= top_k) return;
-  const int c0 = blockIdx.x * kTopkChunk;
-  if (c0 >= V) return;
-  const int c1 = min(V, c0 + kTopkChunk);
+  if (V <= top_k) return;  // every visible cell is selected; no threshold needed
   for (int i = threadIdx.x; i < kBins; i += kTopkThreads) h[i] = 0u;
   __syncthreads();
+  const int c0 = blockIdx.x * kTopkChunk;
+  const int c1 = min(V, c0 + kTopkChunk);
   const float* s = scores + row * ld;
-  for (int c = c0 + threadIdx.x * 4; c < c1; c += kTopkThreads * 4) {
-    if (c + 4 <= c1) {
-      const float4 v = __ldg(reinterpret_cast<const float4*>(s + c));
-      atomicAdd(&h[score_bin(v.x)], 1u);
-      atomicAdd(&h[score_bin(v.y)], 1u);
-      atomicAdd(&h[score_bin(v.z)], 1u);
-      atomicAdd(&h[score_bin(v.w)], 1u);
-    } else {
-      for (int e = c; e < c1; ++e) atomicAdd(&h[score_bin(s[e])], 1u);
+  if (c0 < c1) {
+    for (int c = c0 + threadIdx.x * 4; c < c1; c += kTopkThreads * 4) {
+      if (c + 4 <= c1) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(s + c));
+        atomicAdd(&h[score_bin(v.x)], 1u);
+        atomicAdd(&h[score_bin(v.y)], 1u);
+        atomicAdd(&h[score_bin(v.z)], 1u);
+        atomicAdd(&h[score_bin(v.w)], 1u);
+      } else {
+        for (int e = c; e < c1; ++e) atomicAdd(&h[score_bin(__ldcg(s + e))], 1u);
+      }
     }
   }
   __syncthreads();
   uint32_t* gh = ws.hist + static_cast<size_t>(row) * kBins;
   for (int i = threadIdx.x; i < kBins; i += kTopkThreads)
     if (h[i]) atomicAdd(gh + i, h[i]);
+  uint32_t* ctr = ws.ctr + static_cast<size_t>(row) * kCtrWords;
+  if (last_to_arrive(ctr + kCtrHistDone, gridDim.x, &flag))
+    row_threshold<kTopkThreads>(gh, ctr, static_cast<uint32_t>(top_k), h, scratch, result);
 }
 
-// Append `cell` to a list with one atomic per warp.  Returns nothing; writes
-// only slots below `cap`.
+// Append `cell` to a list with one atomic per warp; only slots below `cap` are written.
 __device__ __forceinline__ void warp_append(bool pred, uint32_t* counter, int32_t* list_ids,
                                             uint2* list_pairs, uint32_t key, int cell, int cap) {
   const uint32_t m = __ballot_sync(0xffffffffu, pred);
@@ -93,115 +140,71 @@ __device__ __forceinline__ void warp_append(bool pred, uint32_t* counter, int32_
   }
 }
 
-// grid: x = chunks, y = rows
-__global__ void __launch_bounds__(kTopkThreads) topk_filter_kernel(const float* __restrict__ scores,
-                                                                   int64_t ld, int vis0, int top_k,
-                                                                   TopkWs ws) {
-  __shared__ uint32_t scratch[33];
-  __shared__ uint32_t result[2];
-  const int row = blockIdx.y;
-  const int V = vis0 + row;
-  if (V <= top_k) return;
-  const int c0 = blockIdx.x * kTopkChunk;
-  if (c0 >= V) return;
-  const int c1 = min(V, c0 + kTopkChunk);
-  uint32_t thr, above;
-  find_threshold_bin<kTopkThreads>(ws.hist + static_cast<size_t>(row) * kBins, kBins,
-                                   static_cast<uint32_t>(top_k), scratch, result, thr, above);
-  const float* s = scores + row * ld;
-  uint32_t* ctr = ws.ctr + static_cast<size_t>(row) * 4;
-  int32_t* sure = ws.sure + static_cast<size_t>(row) * top_k;
-  uint2* cand = ws.cand + static_cast<size_t>(row) * ws.cand_cap;
-  // Every lane walks the chunk in lockstep so the warp-wide ballots line up.
-  for (int base = c0; base < c1; base += kTopkThreads) {
-    const int c = base + threadIdx.x;
-    const bool in = c < c1;
-    const float v = in ? s[c] : 0.f;
-    const uint32_t b = in ? score_bin(v) : 0u;
-    warp_append(in && b > thr, ctr + 0, sure, nullptr, 0u, c, top_k);
-    warp_append(in && b == thr, ctr + 1, nullptr, cand, score_key(v), c, ws.cand_cap);
-  }
-}
+struct SelectSmem {
+  uint32_t h256[256];
+  uint32_t scratch[33];
+  uint32_t result[2];
+  uint32_t flag;
+};
 
-// One CTA per row.  Dynamic shared memory: two bitmaps of win_bits / 32 words
-// (win_bits a multiple of 32, at most kMaxWindowBits).
-__global__ void __launch_bounds__(kFinalThreads) topk_final_kernel(const float* __restrict__ scores,
-                                                                   int64_t ld, int vis0, int top_k,
-                                                                   TopkWs ws, int win_bits,
-                                                                   int32_t* __restrict__ ids) {
-  extern __shared__ uint32_t bitmaps[];
-  uint32_t* selb = bitmaps;
-  uint32_t* eqb = bitmaps + win_bits / 32;
-  __shared__ uint32_t h256[256];
-  __shared__ uint32_t scratch[33];
-  __shared__ uint32_t result[2];
-  const int row = blockIdx.x;
-  const int V = vis0 + row;
+// The exact selection of one row by one CTA of NT threads, once its sure and
+// candidate lists are complete.  `bits` is 2 * win_bits / 32 words of shared memory.
+template <int NT>
+__device__ void final_select(const float* __restrict__ s, int V, int top_k, const uint32_t* ctr,
+                             const int32_t* sure, const uint2* cand, int cand_cap, uint32_t* bits,
+                             int win_bits, SelectSmem& sm, int32_t* __restrict__ out) {
   const int tid = threadIdx.x;
-  int32_t* out = ids + static_cast<size_t>(row) * top_k;
-
-  if (V <= top_k) {  // every visible cell, ascending
-    for (int i = tid; i < top_k; i += kFinalThreads) out[i] = i < V ? i : -1;
-    return;
-  }
-  const float* s = scores + row * ld;
-  uint32_t thr_bin, above;
-  find_threshold_bin<kFinalThreads>(ws.hist + static_cast<size_t>(row) * kBins, kBins,
-                                    static_cast<uint32_t>(top_k), scratch, result, thr_bin,
-                                    above);
-  const uint32_t* ctr = ws.ctr + static_cast<size_t>(row) * 4;
-  const uint32_t n_sure = ctr[0];
-  const uint32_t n_cand_all = ctr[1];
-  const bool overflow = n_cand_all > static_cast<uint32_t>(ws.cand_cap);
+  uint32_t* selb = bits;
+  uint32_t* eqb = bits + win_bits / 32;
+  const uint32_t thr_bin = __ldcg(ctr + kCtrThrBin);
+  const uint32_t n_sure = __ldcg(ctr + kCtrSure);
+  const uint32_t n_cand_all = __ldcg(ctr + kCtrCand);
+  const bool overflow = n_cand_all > static_cast<uint32_t>(cand_cap);
   const int n_src = overflow ? V : static_cast<int>(n_cand_all);
-  const int32_t* sure = ws.sure + static_cast<size_t>(row) * top_k;
-  const uint2* cand = ws.cand + static_cast<size_t>(row) * ws.cand_cap;
-  (void)above;
 
   // Exact threshold key among the candidates: 4 passes of 8 bits.
   uint32_t need = static_cast<uint32_t>(top_k) - n_sure;  // >= 1
   uint32_t prefix = 0u, mask = 0u;
   for (int shift = 24; shift >= 0; shift -= 8) {
-    if (tid < 256) h256[tid] = 0u;
+    for (int i = tid; i < 256; i += NT) sm.h256[i] = 0u;
     __syncthreads();
-    for (int i = tid; i < n_src; i += kFinalThreads) {
+    for (int i = tid; i < n_src; i += NT) {
       uint32_t key;
       if (overflow) {
-        const float v = s[i];
+        const float v = __ldcg(s + i);
         if (score_bin(v) != thr_bin) continue;
         key = score_key(v);
       } else {
-        key = cand[i].x;
+        key = __ldcg(&cand[i].x);
       }
-      if ((key & mask) == prefix) atomicAdd(&h256[(key >> shift) & 255u], 1u);
+      if ((key & mask) == prefix) atomicAdd(&sm.h256[(key >> shift) & 255u], 1u);
     }
     __syncthreads();
     uint32_t digit, cnt_above;
-    find_threshold_bin<kFinalThreads>(h256, 256, need, scratch, result, digit, cnt_above);
+    find_threshold_bin<NT>(sm.h256, 256, need, sm.scratch, sm.result, digit, cnt_above);
     need -= cnt_above;
     prefix |= digit << shift;
     mask |= 255u << shift;
   }
   const uint32_t thr_key = prefix;
-  const uint32_t take_eq = need;  // lowest-index cells with key == thr_key to take
+  const uint32_t take_eq = need;  // lowest-index cells with key == thr_key to keep
 
-  // Bitmap windows over the row's cells, emitted in ascending order.
   uint32_t out_base = 0u, eq_taken = 0u;
   for (int w0 = 0; w0 < V; w0 += win_bits) {
     const int wn = min(win_bits, V - w0);
     const int words = (wn + 31) >> 5;
-    for (int i = tid; i < words; i += kFinalThreads) {
+    for (int i = tid; i < words; i += NT) {
       selb[i] = 0u;
       eqb[i] = 0u;
     }
     __syncthreads();
-    for (uint32_t i = tid; i < n_sure; i += kFinalThreads) {
-      const int c = sure[i] - w0;
+    for (uint32_t i = tid; i < n_sure; i += NT) {
+      const int c = __ldcg(sure + i) - w0;
       if (c >= 0 && c < wn) atomicOr(&selb[c >> 5], 1u << (c & 31));
     }
     if (overflow) {
-      for (int i = w0 + tid; i < w0 + wn; i += kFinalThreads) {
-        const float v = s[i];
+      for (int i = w0 + tid; i < w0 + wn; i += NT) {
+        const float v = __ldcg(s + i);
         if (score_bin(v) != thr_bin) continue;
         const uint32_t key = score_key(v);
         const int c = i - w0;
@@ -209,8 +212,8 @@ __global__ void __launch_bounds__(kFinalThreads) topk_final_kernel(const float* 
         else if (key == thr_key) atomicOr(&eqb[c >> 5], 1u << (c & 31));
       }
     } else {
-      for (int i = tid; i < n_src; i += kFinalThreads) {
-        const uint2 p = cand[i];
+      for (int i = tid; i < n_src; i += NT) {
+        const uint2 p = __ldcg(cand + i);
         const int c = static_cast<int>(p.y) - w0;
         if (c < 0 || c >= wn) continue;
         if (p.x > thr_key) atomicOr(&selb[c >> 5], 1u << (c & 31));
@@ -218,20 +221,18 @@ __global__ void __launch_bounds__(kFinalThreads) topk_final_kernel(const float* 
       }
     }
     __syncthreads();
-    // Each thread owns a contiguous run of words.
-    const int per = (words + kFinalThreads - 1) / kFinalThreads;
+    const int per = (words + NT - 1) / NT;
     const int wb = tid * per, we = min(words, wb + per);
-    // Ties at the threshold: keep the lowest-index take_eq cells overall.
     uint32_t cnt = 0u;
     for (int i = wb; i < we; ++i) cnt += __popc(eqb[i]);
     uint32_t tot;
-    uint32_t rank = eq_taken + block_exclusive_scan<kFinalThreads>(cnt, scratch, tot);
+    uint32_t rank = eq_taken + block_exclusive_scan<NT>(cnt, sm.scratch, tot);
     for (int i = wb; i < we && rank < take_eq; ++i) {
-      uint32_t bits = eqb[i];
-      while (bits && rank < take_eq) {
-        const uint32_t low = bits & (0u - bits);
+      uint32_t b = eqb[i];
+      while (b && rank < take_eq) {
+        const uint32_t low = b & (0u - b);
         selb[i] |= low;
-        bits ^= low;
+        b ^= low;
         ++rank;
       }
     }
@@ -239,20 +240,74 @@ __global__ void __launch_bounds__(kFinalThreads) topk_final_kernel(const float* 
     __syncthreads();
     cnt = 0u;
     for (int i = wb; i < we; ++i) cnt += __popc(selb[i]);
-    uint32_t pos = out_base + block_exclusive_scan<kFinalThreads>(cnt, scratch, tot);
+    uint32_t pos = out_base + block_exclusive_scan<NT>(cnt, sm.scratch, tot);
     for (int i = wb; i < we; ++i) {
-      uint32_t bits = selb[i];
-      while (bits) {
-        const int b = __ffs(bits) - 1;
-        bits &= bits - 1u;
-        if (pos < static_cast<uint32_t>(top_k)) out[pos] = w0 + i * 32 + b;
+      uint32_t b = selb[i];
+      while (b) {
+        const int bit = __ffs(b) - 1;
+        b &= b - 1u;
+        if (pos < static_cast<uint32_t>(top_k)) out[pos] = w0 + i * 32 + bit;
         ++pos;
       }
     }
     out_base += tot;
     __syncthreads();
   }
-  for (uint32_t i = out_base + tid; i < static_cast<uint32_t>(top_k); i += kFinalThreads) out[i] = -1;
+  for (uint32_t i = out_base + tid; i < static_cast<uint32_t>(top_k); i += NT) out[i] = -1;
+}
+
+// grid: x = chunks (of the longest row), y = rows; block kTopkThreads;
+// dynamic smem: two bitmaps of win_bits / 32 words.
+__global__ void __launch_bounds__(kTopkThreads) topk_select_kernel(const float* __restrict__ scores,
+                                                                   int64_t ld, int vis0, int top_k,
+                                                                   TopkWs ws, int win_bits,
+                                                                   int32_t* __restrict__ ids) {
+  extern __shared__ uint32_t bits[];
+  __shared__ SelectSmem sm;
+  griddep_launch();
+  griddep_wait();
+  const int row = blockIdx.y;
+  const int V = vis0 + row;
+  int32_t* out = ids + static_cast<size_t>(row) * top_k;
+  if (V <= top_k) {  // every visible cell, ascending
+    if (blockIdx.x == 0)
+      for (int i = threadIdx.x; i < top_k; i += kTopkThreads) out[i] = i < V ? i : -1;
+    return;
+  }
+  uint32_t* ctr = ws.ctr + static_cast<size_t>(row) * kCtrWords;
+  const float* s = scores + row * ld;
+  int32_t* sure = ws.sure + static_cast<size_t>(row) * top_k;
+  uint2* cand = ws.cand + static_cast<size_t>(row) * ws.cand_cap;
+  const int c0 = blockIdx.x * kTopkChunk;
+  if (c0 < V) {
+    const uint32_t thr = __ldcg(ctr + kCtrThrBin);
+    // all 16 scores of this thread in flight at once
+    float v[16];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int c = c0 + u * (kTopkThreads * 4) + threadIdx.x * 4;
+      if (c + 4 <= V) {
+        const float4 x = __ldcg(reinterpret_cast<const float4*>(s + c));
+        v[4 * u] = x.x; v[4 * u + 1] = x.y; v[4 * u + 2] = x.z; v[4 * u + 3] = x.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[4 * u + e] = (c + e < V) ? __ldcg(s + c + e) : 0.f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int c = c0 + u * (kTopkThreads * 4) + threadIdx.x * 4 + e;
+        const bool in = c < V;
+        const uint32_t b = score_bin(v[4 * u + e]);
+        warp_append(in && b > thr, ctr + kCtrSure, sure, nullptr, 0u, c, top_k);
+        warp_append(in && b == thr, ctr + kCtrCand, nullptr, cand, score_key(v[4 * u + e]), c,
+                    ws.cand_cap);
+      }
+  }
+  if (last_to_arrive(ctr + kCtrSelectDone, gridDim.x, &sm.flag))
+    final_select<kTopkThreads>(s, V, top_k, ctr, sure, cand, ws.cand_cap, bits, win_bits, sm, out);
 }
 
 }  // namespace qsa

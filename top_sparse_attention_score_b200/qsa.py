@@ -40,6 +40,8 @@ SIGNATURES = {
     "qsa_attn": (_I, [_P, _I, _P, _P, _I, _I, _F, _P, _P, _P]),
     "qsa_merge": (_I, [_P, _I, _I, _P, _P]),
     "qsa_topk_static": (_I, [_P, _I64, _I, _I, _I, _P, _P]),
+    "qsa_device_status": (_I, [_P, _P]),
+    "qsa_selftest_wait_timeout": (_I, [_P]),
     "qsa_last_error": (ctypes.c_char_p, []),
     "qsa_launch_count": (ctypes.c_uint64, []),
 }
@@ -233,6 +235,17 @@ def merge(part, out=None, stream=None):
     _check(load().qsa_merge(_ptr(_dev(part, torch.float32, "part")), rows, nsplit,
                             _ptr(_dev(out, torch.float32, "out")), _stream(stream)))
     return out
+
+
+def device_status(stream=None) -> int:
+    """Read and clear the device's status word (0 or QSA_ERR_TIMEOUT); synchronises."""
+    st = ctypes.c_int(0)
+    _check(load().qsa_device_status(ctypes.byref(st), _stream(stream)))
+    return st.value
+
+
+def selftest_wait_timeout(stream=None) -> None:
+    _check(load().qsa_selftest_wait_timeout(_stream(stream)))
 
 
 def launch_count() -> int:
