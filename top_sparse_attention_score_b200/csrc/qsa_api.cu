@@ -101,15 +101,19 @@ int prepare_device() {
   if (cudaGetDevice(&dev) != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaGetDevice failed");
   const uint64_t bit = 1ull << (dev & 63);
   if (done_mask.load() & bit) return QSA_OK;
-  cudaError_t e = cudaFuncSetAttribute(qsa::topk_select_kernel,
+  cudaError_t e = cudaFuncSetAttribute(qsa::topk_final_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        2 * (qsa::kMaxWindowBits / 32) * 4);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(qsa::attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(sizeof(qsa::AttnSmem)));
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(qsa::cluster_select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             64 * qsa::kClusterThreads * 4);
+#define QSA_CLUSTER_SMEM(P)                                                                     \
+  if (e == cudaSuccess)                                                                         \
+    e = cudaFuncSetAttribute(qsa::cluster_select_kernel<P>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             static_cast<int>(qsa::cluster_smem_bytes<P>()));
+  QSA_CLUSTER_SMEM(1) QSA_CLUSTER_SMEM(2) QSA_CLUSTER_SMEM(4) QSA_CLUSTER_SMEM(8)
+  QSA_CLUSTER_SMEM(16) QSA_CLUSTER_SMEM(32) QSA_CLUSTER_SMEM(64)
+#undef QSA_CLUSTER_SMEM
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(qsa::score_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              qsa::kGemmSmemRequest);
@@ -276,18 +280,21 @@ int launch_zero(void* ws, const TopkPlan& p, cudaStream_t s) {
   return launched("topk_zero_kernel");
 }
 
-int launch_select(const float* scores, int64_t ld, int rows, int vis0, int top_k,
-                  const qsa::TopkWs& w, int32_t* ids, cudaStream_t s) {
+int launch_filter_final(const float* scores, int64_t ld, int rows, int vis0, int top_k,
+                        const qsa::TopkWs& w, int32_t* ids, cudaStream_t s) {
   const int vmax = vis0 + rows - 1;
   const dim3 grid((vmax + qsa::kTopkChunk - 1) / qsa::kTopkChunk, rows);
+  launch_pdl(qsa::topk_filter_kernel, grid, dim3(qsa::kTopkThreads), 0, s, scores, ld, vis0, top_k, w);
+  int r = launched("topk_filter_kernel");
+  if (r) return r;
   const int win = std::min(qsa::kMaxWindowBits, static_cast<int>(align_up(vmax, 32)));
   const size_t smem = 2 * static_cast<size_t>(win / 32) * 4;
-  launch_pdl(qsa::topk_select_kernel, grid, dim3(qsa::kTopkThreads), smem, s, scores, ld, vis0, top_k,
+  launch_pdl(qsa::topk_final_kernel, dim3(rows), dim3(qsa::kFinalThreads), smem, s, scores, ld, vis0, top_k,
              w, win, ids);
-  return launched("topk_select_kernel");
+  return launched("topk_final_kernel");
 }
 
-// Selection over given scores: zero, histogram (+ thresholds), select.
+// Selection over given scores: zero, histogram (+ thresholds), filter, final.
 int launch_topk(const float* scores, int64_t ld, int rows, int vis0, int top_k, void* ws,
                 const TopkPlan& p, int32_t* ids, cudaStream_t s) {
   const qsa::TopkWs w = topk_ws(ws, p);
@@ -297,7 +304,7 @@ int launch_topk(const float* scores, int64_t ld, int rows, int vis0, int top_k, 
   const dim3 grid((vmax + qsa::kTopkChunk - 1) / qsa::kTopkChunk, rows);
   launch_pdl(qsa::topk_hist_kernel, grid, dim3(qsa::kTopkThreads), 0, s, scores, ld, vis0, top_k, w);
   if ((r = launched("topk_hist_kernel"))) return r;
-  return launch_select(scores, ld, rows, vis0, top_k, w, ids, s);
+  return launch_filter_final(scores, ld, rows, vis0, top_k, w, ids, s);
 }
 
 // Selection by one 8-CTA cluster per row (rows of at most 8 x 512 x 64 cells).
@@ -307,7 +314,7 @@ int launch_cluster_select_per(const float* scores, int64_t ld, int rows, int vis
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(qsa::kClusterCtas, rows);
   cfg.blockDim = dim3(qsa::kClusterThreads);
-  cfg.dynamicSmemBytes = PER > qsa::kClusterRegPer ? static_cast<size_t>(PER) * qsa::kClusterThreads * 4 : 0;
+  cfg.dynamicSmemBytes = qsa::cluster_smem_bytes<PER>();
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -338,11 +345,12 @@ int launch_cluster_select(const float* scores, int64_t ld, int rows, int vis0, i
   return launch_cluster_select_per<64>(scores, ld, rows, vis0, top_k, ids, s);
 }
 
-// The selection used by qsa_topk and the whole-step calls: one cluster per row
-// when the rows fit one, else the multi-kernel path through the workspace.
+// The selection used by qsa_topk and the whole-step calls.  Decode-sized calls
+// (a few rows, latency-bound) take one cluster per row; larger calls spread each
+// row over many CTAs through the workspace, which keeps every SM busy.
 int launch_selection(const float* scores, int64_t ld, int rows, int vis0, int top_k, void* ws,
                      const TopkPlan& p, int32_t* ids, cudaStream_t s) {
-  if (vis0 + rows - 1 <= kClusterMaxCells)
+  if (rows <= QSA_MAX_DECODE && vis0 + rows - 1 <= kClusterMaxCells)
     return launch_cluster_select(scores, ld, rows, vis0, top_k, ids, s);
   return launch_topk(scores, ld, rows, vis0, top_k, ws, p, ids, s);
 }

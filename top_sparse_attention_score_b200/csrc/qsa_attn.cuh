@@ -88,7 +88,7 @@ __device__ __forceinline__ void attn_issue(AttnStage& st, const AttnArgs& a, con
 }
 
 // grid: (nsplit, 2, rows); block: 128 threads; dynamic smem: sizeof(AttnSmem).
-__global__ void __launch_bounds__(128) attn_kernel(AttnArgs a) {
+__global__ void __launch_bounds__(128, 4) attn_kernel(AttnArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   AttnSmem& sm = *reinterpret_cast<AttnSmem*>(smem_raw);
   const int split = blockIdx.x, kvh = blockIdx.y, row = blockIdx.z;

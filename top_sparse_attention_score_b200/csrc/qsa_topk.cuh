@@ -10,14 +10,14 @@
 //              memory and flushed with atomics -- either fused into the decode
 //              score kernel or by topk_hist_kernel.  The CTA that finishes last
 //              (a fence and a counter, no waiting) finds each row's threshold bin.
-//   select     topk_select_kernel: each CTA appends the cells of its chunk above
+//   filter     topk_filter_kernel: each CTA appends the cells of its chunk above
 //              the threshold bin to the row's "sure" list and the cells in it, with
-//              their full 32-bit keys, to the "candidate" list.  The CTA of the row
-//              that finishes last then radix-selects the exact 32-bit threshold key
-//              among the candidates (four 8-bit passes), keeps the lowest-index
-//              cells among equal keys, and writes the ids in ascending order by
-//              compacting a bitmap of the row's cells.
-// A candidate list that overflows its capacity is not lost: the last CTA then
+//              their full 32-bit keys, to the "candidate" list.
+//   final      topk_final_kernel, one CTA per row: radix-selects the exact 32-bit
+//              threshold key among the candidates (four 8-bit passes), keeps the
+//              lowest-index cells among equal keys, and writes the ids in ascending
+//              order by compacting a bitmap of the row's cells.
+// A candidate list that overflows its capacity is not lost: the final CTA then
 // re-reads the score row itself for that bin.
 #pragma once
 
@@ -25,8 +25,8 @@
 
 namespace qsa {
 
-constexpr int kTopkChunk = 4096;    // scores per hist/select CTA
-constexpr int kTopkThreads = 256;   // hist/select block
+constexpr int kTopkChunk = 4096;    // scores per hist/filter CTA
+constexpr int kTopkThreads = 256;   // hist/filter block
 constexpr int kMaxWindowBits = 1 << 18;  // cells per bitmap window (two 32 KB bitmaps)
 
 // Per-row counters, zeroed before every use.
@@ -80,7 +80,7 @@ __device__ __forceinline__ bool last_to_arrive(uint32_t* counter, uint32_t total
 }
 
 // grid: x = chunks, y = rows
-__global__ void __launch_bounds__(kTopkThreads) topk_hist_kernel(const float* __restrict__ scores,
+__global__ void __launch_bounds__(kTopkThreads, 8) topk_hist_kernel(const float* __restrict__ scores,
                                                                  int64_t ld, int vis0, int top_k,
                                                                  TopkWs ws) {
   __shared__ uint32_t h[kBins];
@@ -97,20 +97,26 @@ __global__ void __launch_bounds__(kTopkThreads) topk_hist_kernel(const float* __
   for (int i = threadIdx.x; i < kBins; i += kTopkThreads) h[i] = 0u;
   __syncthreads();
   const int c0 = blockIdx.x * kTopkChunk;
-  const int c1 = min(V, c0 + kTopkChunk);
   const float* s = scores + row * ld;
-  if (c0 < c1) {
-    for (int c = c0 + threadIdx.x * 4; c < c1; c += kTopkThreads * 4) {
-      if (c + 4 <= c1) {
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(s + c));
-        atomicAdd(&h[score_bin(v.x)], 1u);
-        atomicAdd(&h[score_bin(v.y)], 1u);
-        atomicAdd(&h[score_bin(v.z)], 1u);
-        atomicAdd(&h[score_bin(v.w)], 1u);
+  if (c0 < V) {
+    // all 16 scores of this thread in flight at once
+    float v[16];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int c = c0 + u * (kTopkThreads * 4) + threadIdx.x * 4;
+      if (c + 4 <= V) {
+        const float4 x = __ldcg(reinterpret_cast<const float4*>(s + c));
+        v[4 * u] = x.x; v[4 * u + 1] = x.y; v[4 * u + 2] = x.z; v[4 * u + 3] = x.w;
       } else {
-        for (int e = c; e < c1; ++e) atomicAdd(&h[score_bin(__ldcg(s + e))], 1u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[4 * u + e] = (c + e < V) ? __ldcg(s + c + e) : 0.f;
       }
     }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (c0 + u * (kTopkThreads * 4) + threadIdx.x * 4 + e < V) atomicAdd(&h[score_bin(v[4 * u + e])], 1u);
   }
   __syncthreads();
   uint32_t* gh = ws.hist + static_cast<size_t>(row) * kBins;
@@ -162,10 +168,46 @@ __device__ void final_select(const float* __restrict__ s, int V, int top_k, cons
   const bool overflow = n_cand_all > static_cast<uint32_t>(cand_cap);
   const int n_src = overflow ? V : static_cast<int>(n_cand_all);
 
-  // Exact threshold key among the candidates: 4 passes of 8 bits.
+  // Bits every candidate shares need no radix pass (they all sit in one coarse
+  // bin, so the top byte is usually common): AND and OR of the candidate keys.
+  uint32_t k_and = 0xffffffffu, k_or = 0u;
+  for (int i = tid; i < n_src; i += NT) {
+    uint32_t key;
+    if (overflow) {
+      const float v = __ldcg(s + i);
+      if (score_bin(v) != thr_bin) continue;
+      key = score_key(v);
+    } else {
+      key = __ldcg(&cand[i].x);
+    }
+    k_and &= key;
+    k_or |= key;
+  }
+  k_and = __reduce_and_sync(0xffffffffu, k_and);
+  k_or = __reduce_or_sync(0xffffffffu, k_or);
+  if (tid == 0) {
+    sm.result[0] = 0xffffffffu;
+    sm.result[1] = 0u;
+  }
+  __syncthreads();
+  if ((tid & 31) == 0) {
+    atomicAnd(&sm.result[0], k_and);
+    atomicOr(&sm.result[1], k_or);
+  }
+  __syncthreads();
+  const uint32_t same = ~(sm.result[0] ^ sm.result[1]);
+  const uint32_t common = sm.result[1];
+  __syncthreads();
+  int top = 31;
+  while (top >= 0 && ((same >> top) & 1u)) --top;  // highest differing bit, -1 if none
+  uint32_t mask = top >= 31 ? 0u : (top < 0 ? 0xffffffffu : ~((2u << top) - 1u));
+  uint32_t prefix = common & mask;
+
+  // Exact threshold key among the candidates: 8-bit passes over the differing bits.
   uint32_t need = static_cast<uint32_t>(top_k) - n_sure;  // >= 1
-  uint32_t prefix = 0u, mask = 0u;
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  while (top >= 0) {
+    const int shift = top >= 7 ? top - 7 : 0;
+    const uint32_t width_mask = (2u << (top - shift)) - 1u;
     for (int i = tid; i < 256; i += NT) sm.h256[i] = 0u;
     __syncthreads();
     for (int i = tid; i < n_src; i += NT) {
@@ -177,14 +219,15 @@ __device__ void final_select(const float* __restrict__ s, int V, int top_k, cons
       } else {
         key = __ldcg(&cand[i].x);
       }
-      if ((key & mask) == prefix) atomicAdd(&sm.h256[(key >> shift) & 255u], 1u);
+      if ((key & mask) == prefix) atomicAdd(&sm.h256[(key >> shift) & width_mask], 1u);
     }
     __syncthreads();
     uint32_t digit, cnt_above;
     find_threshold_bin<NT>(sm.h256, 256, need, sm.scratch, sm.result, digit, cnt_above);
     need -= cnt_above;
     prefix |= digit << shift;
-    mask |= 255u << shift;
+    mask |= width_mask << shift;
+    top = shift - 1;
   }
   const uint32_t thr_key = prefix;
   const uint32_t take_eq = need;  // lowest-index cells with key == thr_key to keep
@@ -256,9 +299,54 @@ __device__ void final_select(const float* __restrict__ s, int V, int top_k, cons
   for (uint32_t i = out_base + tid; i < static_cast<uint32_t>(top_k); i += NT) out[i] = -1;
 }
 
-// grid: x = chunks (of the longest row), y = rows; block kTopkThreads;
-// dynamic smem: two bitmaps of win_bits / 32 words.
-__global__ void __launch_bounds__(kTopkThreads) topk_select_kernel(const float* __restrict__ scores,
+// grid: x = chunks (of the longest row), y = rows; block kTopkThreads.
+// Appends each chunk's cells above the threshold bin to the sure list and the
+// cells in it (with their 32-bit keys) to the candidate list.
+__global__ void __launch_bounds__(kTopkThreads, 8) topk_filter_kernel(const float* __restrict__ scores,
+                                                                   int64_t ld, int vis0, int top_k,
+                                                                   TopkWs ws) {
+  griddep_launch();
+  griddep_wait();
+  const int row = blockIdx.y;
+  const int V = vis0 + row;
+  if (V <= top_k) return;
+  const int c0 = blockIdx.x * kTopkChunk;
+  if (c0 >= V) return;
+  uint32_t* ctr = ws.ctr + static_cast<size_t>(row) * kCtrWords;
+  const float* s = scores + row * ld;
+  int32_t* sure = ws.sure + static_cast<size_t>(row) * top_k;
+  uint2* cand = ws.cand + static_cast<size_t>(row) * ws.cand_cap;
+  const uint32_t thr = __ldcg(ctr + kCtrThrBin);
+  // all 16 scores of this thread in flight at once
+  float v[16];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int c = c0 + u * (kTopkThreads * 4) + threadIdx.x * 4;
+    if (c + 4 <= V) {
+      const float4 x = __ldcg(reinterpret_cast<const float4*>(s + c));
+      v[4 * u] = x.x; v[4 * u + 1] = x.y; v[4 * u + 2] = x.z; v[4 * u + 3] = x.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[4 * u + e] = (c + e < V) ? __ldcg(s + c + e) : 0.f;
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int c = c0 + u * (kTopkThreads * 4) + threadIdx.x * 4 + e;
+      const bool in = c < V;
+      const uint32_t b = score_bin(v[4 * u + e]);
+      warp_append(in && b > thr, ctr + kCtrSure, sure, nullptr, 0u, c, top_k);
+      warp_append(in && b == thr, ctr + kCtrCand, nullptr, cand, score_key(v[4 * u + e]), c, ws.cand_cap);
+    }
+}
+
+constexpr int kFinalThreads = 1024;
+
+// One CTA per row once the lists are complete; dynamic smem: two bitmaps of
+// win_bits / 32 words.
+__global__ void __launch_bounds__(kFinalThreads) topk_final_kernel(const float* __restrict__ scores,
                                                                    int64_t ld, int vis0, int top_k,
                                                                    TopkWs ws, int win_bits,
                                                                    int32_t* __restrict__ ids) {
@@ -266,48 +354,17 @@ __global__ void __launch_bounds__(kTopkThreads) topk_select_kernel(const float* 
   __shared__ SelectSmem sm;
   griddep_launch();
   griddep_wait();
-  const int row = blockIdx.y;
+  const int row = blockIdx.x;
   const int V = vis0 + row;
   int32_t* out = ids + static_cast<size_t>(row) * top_k;
   if (V <= top_k) {  // every visible cell, ascending
-    if (blockIdx.x == 0)
-      for (int i = threadIdx.x; i < top_k; i += kTopkThreads) out[i] = i < V ? i : -1;
+    for (int i = threadIdx.x; i < top_k; i += kFinalThreads) out[i] = i < V ? i : -1;
     return;
   }
-  uint32_t* ctr = ws.ctr + static_cast<size_t>(row) * kCtrWords;
-  const float* s = scores + row * ld;
-  int32_t* sure = ws.sure + static_cast<size_t>(row) * top_k;
-  uint2* cand = ws.cand + static_cast<size_t>(row) * ws.cand_cap;
-  const int c0 = blockIdx.x * kTopkChunk;
-  if (c0 < V) {
-    const uint32_t thr = __ldcg(ctr + kCtrThrBin);
-    // all 16 scores of this thread in flight at once
-    float v[16];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int c = c0 + u * (kTopkThreads * 4) + threadIdx.x * 4;
-      if (c + 4 <= V) {
-        const float4 x = __ldcg(reinterpret_cast<const float4*>(s + c));
-        v[4 * u] = x.x; v[4 * u + 1] = x.y; v[4 * u + 2] = x.z; v[4 * u + 3] = x.w;
-      } else {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) v[4 * u + e] = (c + e < V) ? __ldcg(s + c + e) : 0.f;
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int c = c0 + u * (kTopkThreads * 4) + threadIdx.x * 4 + e;
-        const bool in = c < V;
-        const uint32_t b = score_bin(v[4 * u + e]);
-        warp_append(in && b > thr, ctr + kCtrSure, sure, nullptr, 0u, c, top_k);
-        warp_append(in && b == thr, ctr + kCtrCand, nullptr, cand, score_key(v[4 * u + e]), c,
-                    ws.cand_cap);
-      }
-  }
-  if (last_to_arrive(ctr + kCtrSelectDone, gridDim.x, &sm.flag))
-    final_select<kTopkThreads>(s, V, top_k, ctr, sure, cand, ws.cand_cap, bits, win_bits, sm, out);
+  final_select<kFinalThreads>(scores + row * ld, V, top_k, ws.ctr + static_cast<size_t>(row) * kCtrWords,
+                              ws.sure + static_cast<size_t>(row) * top_k,
+                              ws.cand + static_cast<size_t>(row) * ws.cand_cap, ws.cand_cap, bits, win_bits,
+                              sm, out);
 }
 
 }  // namespace qsa

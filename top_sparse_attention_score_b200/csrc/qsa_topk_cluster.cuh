@@ -2,22 +2,28 @@
 //
 // Same result as qsa_topk.cuh (the top_k cells of largest score, equal scores to
 // the lower index, ascending ids; qsa_topk of "opus r15 track A: prompt_chunk wave
-// zipping, ...", what changed, item 1), organised around Blackwell's clusters:
+// zipping, ...", what changed, item 1), organised around Blackwell clusters for the
+// latency of a decode step:
 //
-//   * a cluster of 8 CTAs x 512 threads owns one row; CTA r holds the scores of
-//     cells [r * chunk, (r + 1) * chunk) in registers, read once from L2/HBM;
-//   * the 2048-bin coarse histogram (fp16-key bins, as in qsa_topk.cuh) is built
-//     in each CTA's shared memory and reduced across the cluster through
-//     distributed shared memory: CTA r sums bin slice r of all eight, then every
-//     CTA finds the threshold bin from the eight slice totals;
-//   * four 8-bit radix passes over the threshold bin's full 32-bit keys find the
-//     exact k-th key; each pass is one cluster barrier (per-CTA 256-bin counts,
-//     double-buffered, summed by every CTA);
-//   * each CTA marks its selected cells (and the lowest-index ties) in a bitmap
-//     of its own contiguous range and writes them in ascending order at an
-//     offset summed from the other CTAs' counts.
-// No global atomics, no counters to clear, no candidate lists: only hardware
-// cluster barriers (which need no timeout: every CTA of a cluster is resident).
+//   * a cluster of 8 CTAs x 512 threads owns one row; CTA r holds the order-
+//     preserving keys of cells [r * chunk, (r + 1) * chunk), read once from L2/HBM,
+//     and their coarse bins (the top 10 bits of the key of the score's fp16
+//     rounding, so a higher bin always means a strictly larger score);
+//   * each CTA counts its bins in shared memory (two 16-bit counts per word);
+//     after one cluster barrier every CTA sums all eight through distributed
+//     shared memory and finds the threshold bin itself;
+//   * each CTA lists its cells in the threshold bin (typically a few hundred in
+//     the row); after a second barrier every CTA gathers all lists and one warp
+//     radix-selects the exact k-th key over the bits the candidates do not share,
+//     and derives every CTA's output offset from the gathered lists;
+//   * each CTA marks its selected cells (and the lowest-index ties) in a bitmap of
+//     its own contiguous range and writes them in ascending order.  A split
+//     arrive/wait cluster barrier keeps every CTA's shared memory alive until the
+//     others finished reading it, without a final stall.
+// If the candidates overflow the gather buffers, every CTA of the cluster takes
+// the same slower path: the radix passes run distributed, one cluster barrier each.
+// Only hardware cluster barriers synchronise (all CTAs of a cluster are
+// co-resident): no global atomics, nothing to clear between calls.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -28,39 +34,104 @@ namespace qsa {
 
 constexpr int kClusterCtas = 8;
 constexpr int kClusterThreads = 512;
-constexpr int kClusterSlice = kBins / kClusterCtas;  // 256 bins reduced by each CTA
+constexpr int kClusterRegPer = 16;       // keys per thread kept in registers; beyond, in shared memory
+constexpr int kClusterBins = 1024;       // coarse bins of the cluster histogram
+constexpr int kClusterCandCap = 2048;    // candidates one CTA can list
+constexpr int kClusterGatherCap = 4096;  // candidates a CTA can gather from the whole cluster
 
-// Scores per thread held in registers up to this many; beyond, in shared memory.
-constexpr int kClusterRegPer = 32;
+// Coarse bin of an order-preserving key (score_key): the top 10 bits of the
+// order-preserving key of the score's fp16 rounding.
+__device__ __forceinline__ uint32_t cluster_bin(uint32_t key) {
+  const uint32_t bits = (key & 0x80000000u) ? (key ^ 0x80000000u) : ~key;
+  return score_bin(__uint_as_float(bits)) >> 1;
+}
 
-// grid (8, rows), cluster (8, 1, 1), block 512.  PER scores per thread: the
-// cluster covers 8 * 512 * PER cells, at least the longest row.  For PER above
-// kClusterRegPer the CTA's scores live in dynamic shared memory (PER * 512 floats).
+// One warp, 256 bins counted from the highest: the bin where the running count
+// first reaches k, and the count strictly above it (returned in every lane).
+__device__ __forceinline__ void warp_threshold_256(const uint32_t* h, uint32_t k, uint32_t& bin,
+                                                   uint32_t& above) {
+  const int lane = threadIdx.x & 31;
+  const int hi = 255 - 8 * lane;
+  uint32_t local = 0u;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) local += h[hi - i];
+  uint32_t incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const uint32_t before = incl - local;
+  const uint32_t m = __ballot_sync(0xffffffffu, before < k && incl >= k);
+  const int f = m ? __ffs(m) - 1 : 31;
+  uint32_t b = 0u, ab = 0u;
+  if (lane == f) {
+    uint32_t run = before;
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t c = h[hi - i];
+      if (run + c >= k) {
+        b = static_cast<uint32_t>(hi - i);
+        ab = run;
+        break;
+      }
+      run += c;
+    }
+  }
+  bin = __shfl_sync(0xffffffffu, b, f);
+  above = __shfl_sync(0xffffffffu, ab, f);
+}
+
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+
+template <int PER>
+struct ClusterSmem {
+  static constexpr int kWords = kClusterThreads * PER / 32;
+  uint32_t hist[kClusterBins / 2];    // two 16-bit counts per word
+  uint32_t tot[kClusterBins];
+  uint2 cand[kClusterCandCap];        // (key, local index)
+  uint32_t gkey[kClusterGatherCap];
+  uint32_t gcell[kClusterGatherCap];  // q * chunk + local index
+  uint32_t selb[kWords];
+  uint32_t eqb[kWords];
+  uint32_t radix[2][256];
+  uint32_t tmp256[256];
+  uint32_t pub[4];                    // published: sure count, candidate count, selected count, tie count
+  uint32_t q_sure[kClusterCtas], q_cand[kClusterCtas], q_sel[kClusterCtas], q_eq[kClusterCtas];
+  uint32_t q_off[kClusterCtas];
+  uint32_t cand_n, sure_n, misc[4];
+  uint32_t scratch[33];
+  uint32_t result[2];
+};
+
+template <int PER>
+constexpr size_t cluster_smem_bytes() {
+  return sizeof(ClusterSmem<PER>) + (PER > kClusterRegPer ? static_cast<size_t>(PER) * kClusterThreads * 4 : 0);
+}
+
+// grid (8, rows), cluster (8, 1, 1), block 512, dynamic smem cluster_smem_bytes<PER>().
+// PER cells per thread: the cluster covers 8 * 512 * PER cells, at least the longest row.
 template <int PER>
 __global__ void __launch_bounds__(kClusterThreads) cluster_select_kernel(const float* __restrict__ scores,
                                                                          int64_t ld, int vis0, int top_k,
                                                                          int32_t* __restrict__ ids) {
   namespace cg = cooperative_groups;
   constexpr bool kInSmem = PER > kClusterRegPer;
-  extern __shared__ float sv[];
   constexpr int NT = kClusterThreads;
   constexpr int CHUNK = NT * PER;
   constexpr int WORDS = CHUNK / 32;
-  __shared__ uint32_t hist[kBins];
-  __shared__ uint32_t slice[kClusterSlice];
-  __shared__ uint32_t radix[2][256];
-  __shared__ uint32_t tmp256[256];
-  __shared__ uint32_t selb[WORDS];
-  __shared__ uint32_t eqb[WORDS];
-  __shared__ uint32_t slice_total;
-  __shared__ uint32_t counts[2];  // published: selected cells without ties, cells tied at the threshold
-  __shared__ uint32_t tots[kClusterCtas];
-  __shared__ uint32_t scratch[33];
-  __shared__ uint32_t result[2];
+  extern __shared__ __align__(16) unsigned char csm_raw[];
+  ClusterSmem<PER>& sm = *reinterpret_cast<ClusterSmem<PER>*>(csm_raw);
+  uint32_t* skeys = reinterpret_cast<uint32_t*>(csm_raw + sizeof(ClusterSmem<PER>));
 
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
   const int tid = threadIdx.x;
+  const int lane = tid & 31;
   griddep_launch();
   griddep_wait();
   const int row = blockIdx.y;
@@ -74,146 +145,272 @@ __global__ void __launch_bounds__(kClusterThreads) cluster_select_kernel(const f
   const int c0 = rank * CHUNK;
   const float* s = scores + row * ld;
 
-  // ---- scores of this CTA's cells (element e of thread t is cell c0 + e * NT + t)
-  float v[kInSmem ? 1 : PER];
-#define QSA_SCORE(e) (kInSmem ? sv[(e) * NT + tid] : v[kInSmem ? 0 : (e)])
+  // ---- keys of this CTA's cells (element e of thread t is cell c0 + e * NT + t)
+  uint32_t key[kInSmem ? 1 : PER];
+  uint32_t binpk[kInSmem ? 1 : (PER + 1) / 2];
+#define QSA_KEY(e) (kInSmem ? skeys[(e) * NT + tid] : key[kInSmem ? 0 : (e)])
+#define QSA_BIN(e) \
+  (kInSmem ? cluster_bin(QSA_KEY(e)) : ((binpk[kInSmem ? 0 : (e) >> 1] >> (16 * ((e) & 1))) & 0xffffu))
+  {
+    float x[PER];
 #pragma unroll
-  for (int e = 0; e < PER; ++e) {
-    const int c = c0 + e * NT + tid;
-    const float x = c < V ? __ldcg(s + c) : 0.f;
-    if constexpr (kInSmem) sv[e * NT + tid] = x;
-    else v[e] = x;
+    for (int e = 0; e < PER; ++e) {
+      const int c = c0 + e * NT + tid;
+      x[e] = c < V ? __ldcg(s + c) : 0.f;
+    }
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      const uint32_t k = score_key(x[e]);
+      if constexpr (kInSmem) {
+        skeys[e * NT + tid] = k;
+      } else {
+        key[e] = k;
+        const uint32_t b = score_bin(x[e]) >> 1;
+        if (e & 1) binpk[e >> 1] |= b << 16;
+        else binpk[e >> 1] = b;
+      }
+    }
   }
-  for (int i = tid; i < kBins; i += NT) hist[i] = 0u;
-  if (tid == 0) slice_total = 0u;
+  for (int i = tid; i < kClusterBins / 2; i += NT) sm.hist[i] = 0u;
+  if (tid == 0) {
+    sm.cand_n = 0u;
+    sm.sure_n = 0u;
+  }
   __syncthreads();
 #pragma unroll
   for (int e = 0; e < PER; ++e)
-    if (c0 + e * NT + tid < V) atomicAdd(&hist[score_bin(QSA_SCORE(e))], 1u);
-  cluster.sync();  // every CTA's histogram is complete
-
-  // ---- reduce bin slice `rank` over the cluster; publish its total
-  if (tid < kClusterSlice) {
-    const int b = rank * kClusterSlice + tid;
-    uint32_t sum = 0u;
-#pragma unroll
-    for (int q = 0; q < kClusterCtas; ++q) sum += cluster.map_shared_rank(hist, q)[b];
-    slice[tid] = sum;
-    atomicAdd(&slice_total, sum);
-  }
-  cluster.sync();  // slices and totals published
-
-  // ---- threshold bin: slices from the highest (rank 7) down
-  if (tid < kClusterCtas) tots[tid] = *cluster.map_shared_rank(&slice_total, tid);
-  __syncthreads();
-  uint32_t above = 0u;
-  int qs = 0;
-  for (int q = kClusterCtas - 1; q >= 0; --q) {
-    if (above + tots[q] >= static_cast<uint32_t>(top_k)) {
-      qs = q;
-      break;
+    if (c0 + e * NT + tid < V) {
+      const uint32_t b = QSA_BIN(e);
+      atomicAdd(&sm.hist[b >> 1], 1u << (16 * (b & 1)));  // at most 32768 cells per CTA: no carry
     }
-    above += tots[q];
-  }
-  if (tid < kClusterSlice) tmp256[tid] = cluster.map_shared_rank(slice, qs)[tid];
-  __syncthreads();
-  uint32_t tb, above_in;
-  find_threshold_bin<NT>(tmp256, kClusterSlice, static_cast<uint32_t>(top_k) - above, scratch, result, tb,
-                         above_in);
-  const uint32_t thr_bin = static_cast<uint32_t>(qs * kClusterSlice) + tb;
-  above += above_in;
+  cluster.sync();  // (1) every CTA's histogram is complete
 
-  // ---- exact threshold key among the cells of the threshold bin: 4 passes of 8 bits
+  // ---- every CTA: the row's histogram (one remote word per CTA and thread) and threshold bin
+  {
+    uint32_t lo = 0u, hi = 0u;
+#pragma unroll
+    for (int q = 0; q < kClusterCtas; ++q) {
+      const uint32_t w = cluster.map_shared_rank(sm.hist, q)[tid];
+      lo += w & 0xffffu;
+      hi += w >> 16;
+    }
+    sm.tot[2 * tid] = lo;
+    sm.tot[2 * tid + 1] = hi;
+  }
+  __syncthreads();
+  uint32_t thr_bin, above;
+  find_threshold_bin<NT>(sm.tot, kClusterBins, static_cast<uint32_t>(top_k), sm.scratch, sm.result, thr_bin,
+                         above);
+
+  // ---- count this CTA's cells above the threshold bin; list the ones in it
+  uint32_t my_sure = 0u;
+#pragma unroll
+  for (int e = 0; e < PER; ++e) {
+    const int li = e * NT + tid;
+    const uint32_t b = QSA_BIN(e);
+    const bool valid = c0 + li < V;
+    my_sure += (valid && b > thr_bin) ? 1u : 0u;
+    const bool is_cand = valid && b == thr_bin;
+    const uint32_t m = __ballot_sync(0xffffffffu, is_cand);
+    if (!m) continue;
+    const int leader = __ffs(m) - 1;
+    uint32_t base = 0u;
+    if (lane == leader) base = atomicAdd(&sm.cand_n, static_cast<uint32_t>(__popc(m)));
+    base = __shfl_sync(0xffffffffu, base, leader);
+    if (is_cand) {
+      const uint32_t slot = base + __popc(m & ((1u << lane) - 1u));
+      if (slot < static_cast<uint32_t>(kClusterCandCap))
+        sm.cand[slot] = make_uint2(QSA_KEY(e), static_cast<uint32_t>(li));
+    }
+  }
+  my_sure = __reduce_add_sync(0xffffffffu, my_sure);
+  if (lane == 0) atomicAdd(&sm.sure_n, my_sure);
+  __syncthreads();
+  if (tid == 0) {
+    sm.pub[0] = sm.sure_n;
+    sm.pub[1] = sm.cand_n;
+  }
+  cluster.sync();  // (2) lists and counts published
+
+  if (tid < kClusterCtas) {
+    const uint32_t* p = cluster.map_shared_rank(sm.pub, tid);
+    sm.q_sure[tid] = p[0];
+    sm.q_cand[tid] = p[1];
+  }
+  __syncthreads();
+  uint32_t total_cand = 0u;
+  bool fast = true;
+#pragma unroll
+  for (int q = 0; q < kClusterCtas; ++q) {
+    if (tid == 0) sm.q_off[q] = total_cand;
+    total_cand += sm.q_cand[q];
+    fast = fast && sm.q_cand[q] <= static_cast<uint32_t>(kClusterCandCap);
+  }
+  fast = fast && total_cand <= static_cast<uint32_t>(kClusterGatherCap);  // the same in every CTA
+  __syncthreads();
+
   uint32_t need = static_cast<uint32_t>(top_k) - above;  // >= 1
   uint32_t prefix = 0u, mask = 0u;
+  if (fast) {
+    // gather every candidate of the row; this CTA reads no remote memory after it
+    for (uint32_t i = tid; i < total_cand; i += NT) {
+      int q = kClusterCtas - 1;
+      while (q > 0 && sm.q_off[q] > i) --q;
+      const uint2 p = cluster.map_shared_rank(sm.cand, q)[i - sm.q_off[q]];
+      sm.gkey[i] = p.x;
+      sm.gcell[i] = static_cast<uint32_t>(q * CHUNK) + p.y;
+    }
+    cluster_arrive();
+    __syncthreads();
+    if (tid < 32) {
+      // warp 0: exact threshold key over the bits the candidates do not all share
+      uint32_t k_and = 0xffffffffu, k_or = 0u;
+      for (uint32_t i = lane; i < total_cand; i += 32) {
+        k_and &= sm.gkey[i];
+        k_or |= sm.gkey[i];
+      }
+      k_and = __reduce_and_sync(0xffffffffu, k_and);
+      k_or = __reduce_or_sync(0xffffffffu, k_or);
+      int top = 31;
+      while (top >= 0 && !(((k_and ^ k_or) >> top) & 1u)) --top;  // highest differing bit, -1 if none
+      uint32_t mk = top >= 31 ? 0u : (top < 0 ? 0xffffffffu : ~((2u << top) - 1u));
+      uint32_t pf = k_or & mk, nd = need;
+      while (top >= 0) {
+        const int shift = top >= 7 ? top - 7 : 0;
+        const uint32_t wm = (2u << (top - shift)) - 1u;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sm.tmp256[lane * 8 + i] = 0u;
+        __syncwarp();
+        for (uint32_t i = lane; i < total_cand; i += 32) {
+          const uint32_t k = sm.gkey[i];
+          if ((k & mk) == pf) atomicAdd(&sm.tmp256[(k >> shift) & wm], 1u);
+        }
+        __syncwarp();
+        uint32_t digit, cnt_above;
+        warp_threshold_256(sm.tmp256, nd, digit, cnt_above);
+        __syncwarp();
+        nd -= cnt_above;
+        pf |= digit << shift;
+        mk |= wm << shift;
+        top = shift - 1;
+      }
+      if (lane < kClusterCtas) {
+        sm.q_sel[lane] = sm.q_sure[lane];
+        sm.q_eq[lane] = 0u;
+      }
+      __syncwarp();
+      for (uint32_t i = lane; i < total_cand; i += 32) {
+        const uint32_t k = sm.gkey[i];
+        const int q = static_cast<int>(sm.gcell[i] / CHUNK);
+        if (k > pf) atomicAdd(&sm.q_sel[q], 1u);
+        else if (k == pf) atomicAdd(&sm.q_eq[q], 1u);
+      }
+      if (lane == 0) {
+        sm.misc[2] = pf;
+        sm.misc[3] = nd;
+      }
+    }
+    __syncthreads();
+    prefix = sm.misc[2];
+    need = sm.misc[3];
+  } else {
+    // distributed radix passes over every CTA's own cells, one cluster barrier each
 #pragma unroll 1
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    uint32_t* h = radix[pass & 1];
-    for (int i = tid; i < 256; i += NT) h[i] = 0u;
-    __syncthreads();
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      uint32_t* h = sm.radix[pass & 1];
+      if (tid < 256) h[tid] = 0u;
+      __syncthreads();
 #pragma unroll
-    for (int e = 0; e < PER; ++e) {
-      if (c0 + e * NT + tid >= V || score_bin(QSA_SCORE(e)) != thr_bin) continue;
-      const uint32_t key = score_key(QSA_SCORE(e));
-      if ((key & mask) == prefix) atomicAdd(&h[(key >> shift) & 255u], 1u);
-    }
-    cluster.sync();  // this pass's counts are complete everywhere
-    if (tid < 256) {
-      uint32_t sum = 0u;
+      for (int e = 0; e < PER; ++e) {
+        if (c0 + e * NT + tid >= V || QSA_BIN(e) != thr_bin) continue;
+        const uint32_t k = QSA_KEY(e);
+        if ((k & mask) == prefix) atomicAdd(&h[(k >> shift) & 255u], 1u);
+      }
+      cluster.sync();
+      if (tid < 256) {
+        uint32_t sum = 0u;
 #pragma unroll
-      for (int q = 0; q < kClusterCtas; ++q) sum += cluster.map_shared_rank(h, q)[tid];
-      tmp256[tid] = sum;
+        for (int q = 0; q < kClusterCtas; ++q) sum += cluster.map_shared_rank(h, q)[tid];
+        sm.tmp256[tid] = sum;
+      }
+      __syncthreads();
+      uint32_t digit, cnt_above;
+      find_threshold_bin<NT>(sm.tmp256, 256, need, sm.scratch, sm.result, digit, cnt_above);
+      need -= cnt_above;
+      prefix |= digit << shift;
+      mask |= 255u << shift;
     }
-    __syncthreads();
-    uint32_t digit, cnt_above;
-    find_threshold_bin<NT>(tmp256, 256, need, scratch, result, digit, cnt_above);
-    need -= cnt_above;
-    prefix |= digit << shift;
-    mask |= 255u << shift;
   }
   const uint32_t thr_key = prefix;
   const uint32_t take_eq = need;  // lowest-index cells with key == thr_key to keep
 
-  // ---- mark this CTA's cells; publish its counts
+  // ---- mark this CTA's cells
   for (int i = tid; i < WORDS; i += NT) {
-    selb[i] = 0u;
-    eqb[i] = 0u;
+    sm.selb[i] = 0u;
+    sm.eqb[i] = 0u;
   }
   __syncthreads();
 #pragma unroll
   for (int e = 0; e < PER; ++e) {
     const int li = e * NT + tid;
     if (c0 + li >= V) continue;
-    const uint32_t b = score_bin(QSA_SCORE(e));
+    const uint32_t b = QSA_BIN(e);
     if (b < thr_bin) continue;
-    const uint32_t key = score_key(QSA_SCORE(e));
-    if (b > thr_bin || key > thr_key) atomicOr(&selb[li >> 5], 1u << (li & 31));
-    else if (key == thr_key) atomicOr(&eqb[li >> 5], 1u << (li & 31));
+    const uint32_t k = QSA_KEY(e);
+    if (b > thr_bin || k > thr_key) atomicOr(&sm.selb[li >> 5], 1u << (li & 31));
+    else if (k == thr_key) atomicOr(&sm.eqb[li >> 5], 1u << (li & 31));
   }
   __syncthreads();
   const int per = (WORDS + NT - 1) / NT;
   const int wb = tid * per, we = min(WORDS, wb + per);
   uint32_t nsel = 0u, neq = 0u;
   for (int i = wb; i < we; ++i) {
-    nsel += __popc(selb[i]);
-    neq += __popc(eqb[i]);
+    nsel += __popc(sm.selb[i]);
+    neq += __popc(sm.eqb[i]);
   }
-  uint32_t tot_sel, tot_eq;
-  const uint32_t sel_rank = block_exclusive_scan<NT>(nsel, scratch, tot_sel);
-  const uint32_t eq_rank = block_exclusive_scan<NT>(neq, scratch, tot_eq);
-  if (tid == 0) {
-    counts[0] = tot_sel;
-    counts[1] = tot_eq;
+  // one scan of both counts (each below 2^16: a CTA holds at most 32768 cells)
+  uint32_t tot_pk;
+  const uint32_t rank_pk = block_exclusive_scan<NT>(nsel | (neq << 16), sm.scratch, tot_pk);
+  const uint32_t sel_rank = rank_pk & 0xffffu, eq_rank = rank_pk >> 16;
+  const uint32_t tot_sel = tot_pk & 0xffffu, tot_eq = tot_pk >> 16;
+  if (!fast) {  // the per-CTA counts come from the CTAs themselves
+    if (tid == 0) {
+      sm.pub[2] = tot_sel;
+      sm.pub[3] = tot_eq;
+    }
+    cluster.sync();
+    if (tid < kClusterCtas) {
+      const uint32_t* p = cluster.map_shared_rank(sm.pub, tid);
+      sm.q_sel[tid] = p[2];
+      sm.q_eq[tid] = p[3];
+    }
+    cluster_arrive();
   }
-  cluster.sync();  // counts published
+  __syncthreads();
 
   // ---- offsets from the lower-ranked CTAs; ties go to the lowest indices first
   uint32_t eq_before = 0u, out_before = 0u;
   for (int q = 0; q < rank; ++q) {
-    const uint32_t* cq = cluster.map_shared_rank(counts, q);
-    const uint32_t qsel = cq[0], qeq = cq[1];
-    const uint32_t qtake = eq_before >= take_eq ? 0u : min(qeq, take_eq - eq_before);
-    out_before += qsel + qtake;
-    eq_before += qeq;
+    const uint32_t qtake = eq_before >= take_eq ? 0u : min(sm.q_eq[q], take_eq - eq_before);
+    out_before += sm.q_sel[q] + qtake;
+    eq_before += sm.q_eq[q];
   }
-  uint32_t my_take = eq_before >= take_eq ? 0u : min(tot_eq, take_eq - eq_before);
-  // my eq bits in ascending order: keep the first my_take
+  const uint32_t my_take = eq_before >= take_eq ? 0u : min(tot_eq, take_eq - eq_before);
   uint32_t r = eq_rank;
   for (int i = wb; i < we && r < my_take; ++i) {
-    uint32_t b = eqb[i];
+    uint32_t b = sm.eqb[i];
     while (b && r < my_take) {
       const uint32_t low = b & (0u - b);
-      selb[i] |= low;
+      sm.selb[i] |= low;
       b ^= low;
       ++r;
     }
   }
-  // ties kept by earlier threads shift this thread's output position
-  const uint32_t tie_before = min(eq_rank, my_take);
+  const uint32_t tie_before = min(eq_rank, my_take);  // ties kept by lower threads
   uint32_t pos = out_before + sel_rank + tie_before;
   for (int i = wb; i < we; ++i) {
-    uint32_t b = selb[i];
+    uint32_t b = sm.selb[i];
     while (b) {
       const int bit = __ffs(b) - 1;
       b &= b - 1u;
@@ -221,8 +418,9 @@ __global__ void __launch_bounds__(kClusterThreads) cluster_select_kernel(const f
       ++pos;
     }
   }
-  cluster.sync();  // no CTA leaves while another may still read its shared memory
-#undef QSA_SCORE
+  cluster_wait();  // every CTA has finished reading this CTA's shared memory
+#undef QSA_KEY
+#undef QSA_BIN
 }
 
 }  // namespace qsa
