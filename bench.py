@@ -312,7 +312,6 @@ def run_cuda(args, spec: Spec):
                 qsa.prefill_chunk(c, spec.pos0, qq, iqq, iww, spec.top_k, wl.scale, ws=ws, out=o,
                                   ids_out=ids)
 
-    steps = args.steps or (3000 if spec.kind == "decode" else 100)
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
@@ -329,6 +328,19 @@ def run_cuda(args, spec: Spec):
         graphs.append(g)
     for i in range(args.warmup):
         graphs[i % ROTATE].replay()
+    torch.cuda.synchronize()
+    if args.steps:
+        steps = args.steps
+    else:  # about two seconds of timed work, so the clock sampler sees the GPU under load
+        probe0, probe1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        probe0.record(stream)
+        for i in range(2 * ROTATE):
+            graphs[i % ROTATE].replay()
+        probe1.record(stream)
+        torch.cuda.synchronize()
+        per_step = probe0.elapsed_time(probe1) / (2 * ROTATE)
+        steps = int(max(20, min(100000, 2000.0 / max(per_step, 1e-3))))
+        steps = int(dist_max(float(steps), world))
     barrier(world)
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

@@ -246,6 +246,17 @@ int launch_score_gemm(const qsa_cache* c, int rows, int ncells, const uint16_t* 
                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (cr != CUDA_SUCCESS) return fail(QSA_ERR_CUDA, "tensor map of the queries: error %d", static_cast<int>(cr));
   }
+  CUtensorMap tout;
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(ncells), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 4};
+    const cuuint32_t box[2] = {32u, static_cast<cuuint32_t>(qsa::kGemmTokens)};
+    const cuuint32_t estr[2] = {1u, 1u};
+    const CUresult cr = encode(&tout, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, scores, dims, strides, box, estr,
+                               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return fail(QSA_ERR_CUDA, "tensor map of the scores: error %d", static_cast<int>(cr));
+  }
   qsa::GemmArgs a;
   a.iw = iw;
   a.scores = scores;
@@ -256,7 +267,7 @@ int launch_score_gemm(const qsa_cache* c, int rows, int ncells, const uint16_t* 
   const int items = ((rows + qsa::kGemmTokens - 1) / qsa::kGemmTokens) *
                     ((ncells + qsa::kGemmCells - 1) / qsa::kGemmCells);
   const dim3 grid(std::max(1, std::min(items, sm_count())));
-  launch_pdl(qsa::score_gemm_kernel, grid, dim3(qsa::kGemmThreads), qsa::kGemmSmemRequest, s, tkey, tiq, a);
+  launch_pdl(qsa::score_gemm_kernel, grid, dim3(qsa::kGemmThreads), qsa::kGemmSmemRequest, s, tkey, tiq, tout, a);
   return launched("score_gemm_kernel");
 }
 

@@ -5,7 +5,7 @@
 //   score[t][c] = sum_h w[t][h] * max(0, sum_d iq[t][h][d] * key[c][d])   (4 heads x 64, fp16)
 // is four [T x 64] x [64 x L] products followed by a ReLU-weighted sum over heads.
 //
-// sm_100a design (one persistent CTA per SM, 10 warps):
+// sm_100a design (one persistent CTA per SM, 19 warps):
 //   * a tile is 128 tokens x 64 cells.  For each head h one tcgen05.mma chain
 //     (M = 128, N = 64, four K = 16 steps) writes D_h = iq_h . key^T into its own
 //     64 TMEM columns, so token t's four head products sit in TMEM lane t at the
@@ -14,8 +14,11 @@
 //     memory while a CTA sweeps its cells; key tiles (64 x 64 fp16 = 8 KB) stream
 //     in through a 4-stage TMA ring, both with the 128-byte swizzle the UMMA
 //     K-major descriptors describe;
-//   * warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs (one thread),
-//     warps 2..9 are the epilogue.  TMEM holds two 256-column accumulators, so
+//   * warp 0 issues TMA loads, warp 1 owns TMEM and issues the MMAs (one
+//     thread), warps 2..17 are the epilogue (four per TMEM lane quadrant, 16
+//     columns each), warp 18 issues TMA stores.  The epilogue writes each score
+//     tile into a double-buffered shared stage in the 128-byte-swizzled layout,
+//     and the stores move whole 128-byte row segments to global memory;  TMEM holds two 256-column accumulators, so
 //     the epilogue of tile i overlaps the MMAs of tile i + 1;
 //   * every wait on an mbarrier is bounded (one second of %globaltimer): on
 //     expiry the CTA records QSA_ERR_TIMEOUT in `status`, every role stops,
@@ -31,14 +34,18 @@ namespace qsa {
 constexpr int kGemmTokens = 128;     // M
 constexpr int kGemmCells = 64;       // N per head
 constexpr int kGemmStages = 4;       // key-tile ring
-constexpr int kGemmEpiWarps = 8;
-constexpr int kGemmThreads = (2 + kGemmEpiWarps) * 32;
+constexpr int kGemmEpiWarps = 16;
+constexpr int kGemmStoreWarp = 2 + kGemmEpiWarps;           // issues the TMA stores
+constexpr int kGemmThreads = (3 + kGemmEpiWarps) * 32;
 constexpr int kGemmABytes = kHI * kGemmTokens * kDI * 2;   // 64 KB
 constexpr int kGemmBBytes = kGemmCells * kDI * 2;           // 8 KB
-constexpr int kGemmSmemBytes = kGemmABytes + kGemmStages * kGemmBBytes + 1024 /*barriers*/ + 1024 /*align*/;
-// Ask for more shared memory than two CTAs could share, so one CTA owns an SM
-// and its TMEM (the CTA allocates all 512 columns).
-constexpr int kGemmSmemRequest = 120 * 1024;
+constexpr int kGemmCHalfBytes = kGemmTokens * 32 * 4;       // 16 KB: 128 rows x 32 fp32 scores
+constexpr int kGemmSmemBytes = kGemmABytes + kGemmStages * kGemmBBytes + 4 * kGemmCHalfBytes +
+                               1024 /*barriers*/ + 1024 /*align*/;
+// More shared memory than two CTAs could share, so one CTA owns an SM and its
+// TMEM (the CTA allocates all 512 columns).
+constexpr int kGemmSmemRequest = kGemmSmemBytes;
+static_assert(kGemmSmemRequest > 114 * 1024, "one GEMM CTA per SM");
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // one second
 constexpr uint32_t kStatusTimeout = 4;                       // QSA_ERR_TIMEOUT
 
@@ -58,6 +65,8 @@ struct __align__(8) GemmBarriers {
   uint64_t a_empty;
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
+  uint64_t stage_full[2];   // epilogue warps wrote a score tile into the staging buffer
+  uint64_t stage_free[2];   // the TMA store finished reading that buffer
   uint64_t drain;
   uint32_t tmem_base;
   uint32_t abort;
@@ -145,6 +154,22 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int x, int y, const void* src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];\n" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(smem_u32(src))
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;\n" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+
 // UMMA shared-memory descriptor: K-major operand rows of 128 bytes with the
 // 128-byte swizzle (8-row atoms of 1024 bytes: leading offset 16 B, stride 1024 B).
 __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
@@ -185,13 +210,15 @@ __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::
 // grid: number of SMs (persistent); block: kGemmThreads; dynamic smem: kGemmSmemRequest.
 __global__ void __launch_bounds__(kGemmThreads, 1)
     score_gemm_kernel(const __grid_constant__ CUtensorMap tmap_key,
-                      const __grid_constant__ CUtensorMap tmap_iq, GemmArgs a) {
+                      const __grid_constant__ CUtensorMap tmap_iq,
+                      const __grid_constant__ CUtensorMap tmap_out, GemmArgs a) {
   extern __shared__ __align__(1024) unsigned char gsm_raw[];
   unsigned char* gsm = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   unsigned char* sA = gsm;                                   // 4 heads x 16 KB
   unsigned char* sB = gsm + kGemmABytes;                     // stages x 8 KB
-  GemmBarriers& gb = *reinterpret_cast<GemmBarriers*>(sB + kGemmStages * kGemmBBytes);
+  unsigned char* sC = sB + kGemmStages * kGemmBBytes;        // 2 buffers x 2 halves x 16 KB
+  GemmBarriers& gb = *reinterpret_cast<GemmBarriers*>(sC + 4 * kGemmCHalfBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntb = (a.T + kGemmTokens - 1) / kGemmTokens;
@@ -211,6 +238,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&gb.acc_full[b], 1);
       mbar_init(&gb.acc_empty[b], kGemmEpiWarps);
+      mbar_init(&gb.stage_full[b], kGemmEpiWarps);
+      mbar_init(&gb.stage_free[b], 1);
     }
     mbar_init(&gb.drain, 1);
     gb.abort = 0u;
@@ -296,16 +325,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_drain_wait(&gb.drain, 0);
     }
     __syncwarp();
+  } else if (warp == kGemmStoreWarp) {
+    // ---------------- TMA stores of the staged score tiles (two 32-column boxes each)
+    if (lane == 0) {
+      for (int it = it0; it < it1; ++it) {
+        const int tb = it / nct, ct = it % nct;
+        const int li = it - it0, sb = li & 1;
+        if (!mbar_wait(&gb.stage_full[sb], (li >> 1) & 1, gb, a.status)) break;
+        for (int h = 0; h < 2; ++h)  // a box past the last column has nothing to write
+          if (ct * kGemmCells + 32 * h < a.ncells)
+            tma_store_2d(&tmap_out, ct * kGemmCells + 32 * h, tb * kGemmTokens,
+                         sC + (sb * 2 + h) * kGemmCHalfBytes);
+        bulk_commit();
+        // the previous tile's buffer is free once its store has read it
+        bulk_wait_read<1>();
+        if (li > 0) mbar_arrive(&gb.stage_free[sb ^ 1]);
+      }
+      bulk_wait_all();  // every store of this CTA has landed in global memory
+    }
+    __syncwarp();
   } else {
-    // ---------------- epilogue: 8 warps; warp w reads TMEM lanes 32 * (w % 4) ...
+    // ---------------- epilogue: 16 warps; warp w reads TMEM lanes 32 * (w % 4) ...
     const int quad = warp & 3;
-    const int half = (warp - 2) >> 2;  // columns [32 * half, 32 * half + 32) of each head
+    const int colq = (warp - 2) >> 2;  // columns [16 * colq, 16 * colq + 16) of each head
+    const int r = quad * 32 + lane;    // tile row of this thread
     int cur_tb = -1;
     float w[kHI] = {0.f, 0.f, 0.f, 0.f};
     for (int it = it0; it < it1; ++it) {
-      const int tb = it / nct, ct = it % nct;
+      const int tb = it / nct;
       const int li = it - it0, buf = li & 1, bround = li >> 1;
-      const int row = tb * kGemmTokens + quad * 32 + lane;
+      const int row = tb * kGemmTokens + r;
       if (tb != cur_tb) {
 #pragma unroll
         for (int h = 0; h < kHI; ++h) w[h] = row < a.T ? __ldg(a.iw + row * kHI + h) : 0.f;
@@ -318,42 +367,43 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       __syncwarp();
       tc_fence_after();
       if (!ok) break;
+      const int col = colq * 16;
+      uint32_t rr[kHI][16];
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const int col = half * 32 + q * 16;
-        uint32_t r[kHI][16];
-#pragma unroll
-        for (int h = 0; h < kHI; ++h)
-          tmem_ld16(tmem + (static_cast<uint32_t>(quad * 32) << 16) +
-                        static_cast<uint32_t>(buf * 256 + h * kGemmCells + col),
-                    r[h]);
-        tmem_ld_wait();
-        float sc[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          float sacc = w[0] * fmaxf(__uint_as_float(r[0][j]), 0.f);
-          sacc = fmaf(w[1], fmaxf(__uint_as_float(r[1][j]), 0.f), sacc);
-          sacc = fmaf(w[2], fmaxf(__uint_as_float(r[2][j]), 0.f), sacc);
-          sc[j] = fmaf(w[3], fmaxf(__uint_as_float(r[3][j]), 0.f), sacc);
-        }
-        const int c = ct * kGemmCells + col;
-        if (row < a.T) {
-          float* dst = a.scores + row * a.ld + c;
-          if (c + 16 <= a.ncells) {
-#pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4)
-              *reinterpret_cast<float4*>(dst + 4 * v4) =
-                  make_float4(sc[4 * v4], sc[4 * v4 + 1], sc[4 * v4 + 2], sc[4 * v4 + 3]);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-              if (c + j < a.ncells) dst[j] = sc[j];
-          }
-        }
-      }
+      for (int h = 0; h < kHI; ++h)
+        tmem_ld16(tmem + (static_cast<uint32_t>(quad * 32) << 16) +
+                      static_cast<uint32_t>(buf * 256 + h * kGemmCells + col),
+                  rr[h]);
+      tmem_ld_wait();
+      // the accumulator is in registers: hand it back to the MMA warp now
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&gb.acc_empty[buf]);
+      float sc[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        float sacc = w[0] * fmaxf(__uint_as_float(rr[0][j]), 0.f);
+        sacc = fmaf(w[1], fmaxf(__uint_as_float(rr[1][j]), 0.f), sacc);
+        sacc = fmaf(w[2], fmaxf(__uint_as_float(rr[2][j]), 0.f), sacc);
+        sc[j] = fmaf(w[3], fmaxf(__uint_as_float(rr[3][j]), 0.f), sacc);
+      }
+      // stage the scores: buffer li & 1, half colq / 2, 128-byte rows with 16-byte
+      // chunk c stored at c ^ (row % 8) (the layout the TMA store's 128-byte swizzle reads)
+      const int sb = li & 1;
+      ok = 1u;
+      if (lane == 0) ok = mbar_wait(&gb.stage_free[sb], ((li >> 1) & 1) ^ 1, gb, a.status) ? 1u : 0u;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      unsigned char* half = sC + (sb * 2 + (colq >> 1)) * kGemmCHalfBytes + r * 128;
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const int chunk = ((colq & 1) * 4 + jj) ^ (r & 7);
+        *reinterpret_cast<float4*>(half + chunk * 16) =
+            make_float4(sc[4 * jj], sc[4 * jj + 1], sc[4 * jj + 2], sc[4 * jj + 3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&gb.stage_full[sb]);
     }
   }
 

@@ -301,10 +301,14 @@ __device__ void final_select(const float* __restrict__ s, int V, int top_k, cons
 
 // grid: x = chunks (of the longest row), y = rows; block kTopkThreads.
 // Appends each chunk's cells above the threshold bin to the sure list and the
-// cells in it (with their 32-bit keys) to the candidate list.
+// cells in it (with their 32-bit keys) to the candidate list.  The CTA counts
+// its cells first and reserves its slots with one global atomic per list, so no
+// warp waits on an atomic round trip per hit.
 __global__ void __launch_bounds__(kTopkThreads, 8) topk_filter_kernel(const float* __restrict__ scores,
-                                                                   int64_t ld, int vis0, int top_k,
-                                                                   TopkWs ws) {
+                                                                      int64_t ld, int vis0, int top_k,
+                                                                      TopkWs ws) {
+  __shared__ uint32_t warp_n[2][kTopkThreads / 32];
+  __shared__ uint32_t base_g[2];
   griddep_launch();
   griddep_wait();
   const int row = blockIdx.y;
@@ -312,6 +316,7 @@ __global__ void __launch_bounds__(kTopkThreads, 8) topk_filter_kernel(const floa
   if (V <= top_k) return;
   const int c0 = blockIdx.x * kTopkChunk;
   if (c0 >= V) return;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t* ctr = ws.ctr + static_cast<size_t>(row) * kCtrWords;
   const float* s = scores + row * ld;
   int32_t* sure = ws.sure + static_cast<size_t>(row) * top_k;
@@ -330,16 +335,56 @@ __global__ void __launch_bounds__(kTopkThreads, 8) topk_filter_kernel(const floa
       for (int e = 0; e < 4; ++e) v[4 * u + e] = (c + e < V) ? __ldcg(s + c + e) : 0.f;
     }
   }
+  // classify: bit e of `up` / `eq` marks element e above / in the threshold bin
+  uint32_t up = 0u, eq = 0u;
 #pragma unroll
-  for (int u = 0; u < 4; ++u)
+  for (int e = 0; e < 16; ++e) {
+    const int c = c0 + (e >> 2) * (kTopkThreads * 4) + threadIdx.x * 4 + (e & 3);
+    if (c >= V) continue;
+    const uint32_t b = score_bin(v[e]);
+    up |= (b > thr ? 1u : 0u) << e;
+    eq |= (b == thr ? 1u : 0u) << e;
+  }
+  const uint32_t nu = __popc(up), ne = __popc(eq);
+  // per-warp exclusive offsets, then per-CTA offsets, then one global atomic per list
+  uint32_t xu = nu, xe = ne;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int c = c0 + u * (kTopkThreads * 4) + threadIdx.x * 4 + e;
-      const bool in = c < V;
-      const uint32_t b = score_bin(v[4 * u + e]);
-      warp_append(in && b > thr, ctr + kCtrSure, sure, nullptr, 0u, c, top_k);
-      warp_append(in && b == thr, ctr + kCtrCand, nullptr, cand, score_key(v[4 * u + e]), c, ws.cand_cap);
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t yu = __shfl_up_sync(0xffffffffu, xu, o);
+    const uint32_t ye = __shfl_up_sync(0xffffffffu, xe, o);
+    if (lane >= o) {
+      xu += yu;
+      xe += ye;
     }
+  }
+  if (lane == 31) {
+    warp_n[0][warp] = xu;
+    warp_n[1][warp] = xe;
+  }
+  __syncthreads();
+  if (threadIdx.x < 2) {
+    uint32_t tot = 0u;
+    for (int w = 0; w < kTopkThreads / 32; ++w) {
+      const uint32_t n = warp_n[threadIdx.x][w];
+      warp_n[threadIdx.x][w] = tot;
+      tot += n;
+    }
+    base_g[threadIdx.x] = tot ? atomicAdd(ctr + (threadIdx.x == 0 ? kCtrSure : kCtrCand), tot) : 0u;
+  }
+  __syncthreads();
+  uint32_t pu = base_g[0] + warp_n[0][warp] + xu - nu;
+  uint32_t pe = base_g[1] + warp_n[1][warp] + xe - ne;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const int c = c0 + (e >> 2) * (kTopkThreads * 4) + threadIdx.x * 4 + (e & 3);
+    if ((up >> e) & 1u) {
+      if (pu < static_cast<uint32_t>(top_k)) sure[pu] = c;
+      ++pu;
+    } else if ((eq >> e) & 1u) {
+      if (pe < static_cast<uint32_t>(ws.cand_cap)) cand[pe] = make_uint2(score_key(v[e]), static_cast<uint32_t>(c));
+      ++pe;
+    }
+  }
 }
 
 constexpr int kFinalThreads = 1024;
