@@ -227,13 +227,15 @@ def _id_lists(seed, rows, cells, k, nvalid):
     return ids
 
 
+# up to 8 rows run the 4-warp attention kernel, more rows the 2-warp one
+@pytest.mark.parametrize("rows", [3, 12])
 @pytest.mark.parametrize("nsplit", [1, 3, 8, 64])
-def test_attn_vs_oracle(gpu, nsplit):
+def test_attn_vs_oracle(gpu, nsplit, rows):
     qsa = gpu
     cells, k = 4096, 512
     wl = synth.make_workload(0, cells=cells)
-    q, _, _ = synth.make_queries(201, 3)
-    ids = _id_lists(202, 3, cells, k, [512, 300, 17])
+    q, _, _ = synth.make_queries(201, rows)
+    ids = _id_lists(202, rows, cells, k, ([512, 300, 17] * 4)[:rows])
     cache = qsa.DeviceCache.from_host(wl.cache, DEV)
     qd = torch.from_numpy(q).to(DEV)
     idd = torch.from_numpy(ids).to(DEV)
@@ -241,12 +243,12 @@ def test_attn_vs_oracle(gpu, nsplit):
     out = res if nsplit == 1 else qsa.merge(res)
     torch.cuda.synchronize()
     out = out.cpu().numpy()
-    for r in range(3):
+    for r in range(rows):
         ref = oracle.attn_row(wl.cache, q[r], ids[r], 1 / 16)
         assert rel_err(out[r], ref) <= OUT_TOL
     if nsplit > 1:
         part = res.cpu().numpy()
-        for r in range(3):
+        for r in range(rows):
             m, l, o = oracle.partials_row(wl.cache, q[r], ids[r], nsplit, 1 / 16)
             pm, pl, po = part[r, :, :, 0], part[r, :, :, 1], part[r, :, :, 2:].astype(np.float64)
             empty = l == 0

@@ -105,8 +105,11 @@ int prepare_device() {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        2 * (qsa::kMaxWindowBits / 32) * 4);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(qsa::attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(sizeof(qsa::AttnSmem)));
+    e = cudaFuncSetAttribute(qsa::attn_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(sizeof(qsa::AttnSmem<4>)));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(qsa::attn_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(sizeof(qsa::AttnSmem<2>)));
 #define QSA_CLUSTER_SMEM(P)                                                                     \
   if (e == cudaSuccess)                                                                         \
     e = cudaFuncSetAttribute(qsa::cluster_select_kernel<P>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
@@ -340,7 +343,9 @@ int launch_cluster_select_per(const float* scores, int64_t ld, int rows, int vis
   return launched("cluster_select_kernel");
 }
 
-constexpr int kClusterMaxCells = qsa::kClusterCtas * qsa::kClusterThreads * 64;
+// Longest row the decode selection gives to one cluster (16 cells per thread); longer
+// rows go through the multi-kernel selection, which spreads them over more SMs.
+constexpr int kClusterMaxCells = qsa::kClusterCtas * qsa::kClusterThreads * 16;
 
 int launch_cluster_select(const float* scores, int64_t ld, int rows, int vis0, int top_k,
                           int32_t* ids, cudaStream_t s) {
@@ -382,7 +387,10 @@ int launch_attn(const qsa_cache* c, int rows, const float* q, const int32_t* ids
   a.scale_log2 = scale * 1.4426950408889634f;
   a.part = part;
   a.out = out;
-  launch_pdl(qsa::attn_kernel, dim3(nsplit, QSA_HKV, rows), dim3(128), sizeof(qsa::AttnSmem), s, a);
+  if (rows <= QSA_MAX_DECODE)
+    launch_pdl(qsa::attn_kernel<4>, dim3(nsplit, QSA_HKV, rows), dim3(128), sizeof(qsa::AttnSmem<4>), s, a);
+  else
+    launch_pdl(qsa::attn_kernel<2>, dim3(nsplit, QSA_HKV, rows), dim3(64), sizeof(qsa::AttnSmem<2>), s, a);
   return launched("attn_kernel");
 }
 

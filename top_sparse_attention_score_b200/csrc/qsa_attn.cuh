@@ -10,10 +10,10 @@
 //  * cells are gathered 32 at a time with cp.async (16-byte copies of whole
 //    256-byte K/V rows and their scales) into a double-buffered shared-memory
 //    ring, so the next block's gathers are in flight while one computes;
-//  * the four warps split the 256 dims: each computes a partial QK^T over its
-//    64 dims (two scale groups), the partials are summed through shared memory
-//    in a fixed order (all warps get bit-equal scores), each warp runs the same
-//    online softmax and accumulates P.V for its own 64 dims;
+//  * two warps split the 256 dims: each computes a partial QK^T over its 128
+//    dims (four scale groups), the two partials are summed through shared memory
+//    in a fixed order (both warps get bit-equal scores), each warp runs the same
+//    online softmax and accumulates P.V for its own 128 dims;
 //  * int8 codes become fp16 exactly (byte-permute with the 0x6400 exponent).  The
 //    per-32 K scale multiplies each 32-dim partial product in fp32 after the
 //    MMA; the per-32 V scale multiplies the fp16 V operand.  Q and P are fp16.
@@ -37,9 +37,12 @@ struct __align__(16) AttnStage {
 
 constexpr int kAttnStages = 2;
 
+// W warps split the 256 dims (W = 4 for the latency of decode, 2 for the
+// throughput of prefill: half the duplicated softmax and score-reduction work).
+template <int W>
 struct AttnSmem {
   AttnStage st[kAttnStages];
-  float4 red[4][4][32];  // [warp][n-tile][lane] partial scores
+  float4 red[W][4][32];  // [warp][n-tile][lane] partial scores
 };
 
 struct AttnArgs {
@@ -58,13 +61,14 @@ struct AttnArgs {
   float* out;         // [rows][24][256] when nsplit == 1
 };
 
+template <int NT>
 __device__ __forceinline__ void attn_issue(AttnStage& st, const AttnArgs& a, const int* rid, int pos0,
                                            int end, int kvh) {
   const int tid = threadIdx.x;
-  // K and V rows: 32 cells x 16 chunks of 16 bytes each, 4 + 4 per thread.
+  // K and V rows: 32 cells x 16 chunks of 16 bytes each, 512 / NT + 512 / NT per thread.
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int chunk = tid + 128 * u;
+  for (int u = 0; u < 512 / NT; ++u) {
+    const int chunk = tid + NT * u;
     const int i = chunk >> 4, part = chunk & 15;
     const int p = pos0 + i;
     int cell = p < end ? __ldg(rid + p) : -1;
@@ -74,7 +78,7 @@ __device__ __forceinline__ void attn_issue(AttnStage& st, const AttnArgs& a, con
     cp_async16(st.k + i * kAttnKStride + part * 16, a.k + row, ok);
     cp_async16(st.v + i * kAttnVStride + part * 16, a.v + row, ok);
   }
-  if (tid < 2 * kAttnCells) {
+  if (tid < 2 * kAttnCells) {  // scales: 64 rows of 16 bytes
     const int i = tid & 31;
     const int p = pos0 + i;
     int cell = p < end ? __ldg(rid + p) : -1;
@@ -87,10 +91,12 @@ __device__ __forceinline__ void attn_issue(AttnStage& st, const AttnArgs& a, con
   }
 }
 
-// grid: (nsplit, 2, rows); block: 128 threads; dynamic smem: sizeof(AttnSmem).
-__global__ void __launch_bounds__(128, 4) attn_kernel(AttnArgs a) {
+// grid: (nsplit, 2, rows); block: 32 * W threads; dynamic smem: sizeof(AttnSmem<W>).
+template <int W>
+__global__ void __launch_bounds__(32 * W) attn_kernel(AttnArgs a) {
+  constexpr int NT = 32 * W;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  AttnSmem& sm = *reinterpret_cast<AttnSmem*>(smem_raw);
+  AttnSmem<W>& sm = *reinterpret_cast<AttnSmem<W>*>(smem_raw);
   const int split = blockIdx.x, kvh = blockIdx.y, row = blockIdx.z;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
@@ -100,19 +106,20 @@ __global__ void __launch_bounds__(128, 4) attn_kernel(AttnArgs a) {
   const int nblk = (end - beg + kAttnCells - 1) / kAttnCells;
   griddep_launch();
 
-  // Q fragments for this warp's two scale groups (dims [64w, 64w+64)), prescaled.
+  // Q fragments for this warp's four scale groups (dims [128w, 128w+128)), prescaled.
   // Within group qg, thread t covers dims 32qg + 8t + 4s + {0..3} in sub-step s:
   // k-index 2t,2t+1 <-> +0,+1 and 2t+8,2t+9 <-> +2,+3 (the same map as the K loads).
-  uint32_t aq[2][2][4];
+  constexpr int GW = kNG / W;  // scale groups (32 dims each) per warp
+  uint32_t aq[GW][2][4];
   {
     const float* q0 = a.q + (static_cast<size_t>(row) * kHQ + kvh * kQPerKV + g) * kD;
     const float* q8 = q0 + 8 * kD;
     const bool has8 = g + 8 < kQPerKV;
 #pragma unroll
-    for (int gi = 0; gi < 2; ++gi)
+    for (int gi = 0; gi < GW; ++gi)
 #pragma unroll
       for (int s = 0; s < 2; ++s) {
-        const int d0 = 32 * (2 * warp + gi) + 8 * t + 4 * s;
+        const int d0 = 32 * (GW * warp + gi) + 8 * t + 4 * s;
         const float4 x = __ldg(reinterpret_cast<const float4*>(q0 + d0));
         const float sl = a.scale_log2;
         aq[gi][s][0] = pack_half2(x.x * sl, x.y * sl);
@@ -132,15 +139,15 @@ __global__ void __launch_bounds__(128, 4) attn_kernel(AttnArgs a) {
   griddep_wait();
 #pragma unroll
   for (int st = 0; st < kAttnStages - 1; ++st) {
-    if (st < nblk) attn_issue(sm.st[st], a, rid, beg + st * kAttnCells, end, kvh);
+    if (st < nblk) attn_issue<NT>(sm.st[st], a, rid, beg + st * kAttnCells, end, kvh);
     cp_async_commit();
   }
 
   float m_run[2] = {-INFINITY, -INFINITY};
   float l_run[2] = {0.f, 0.f};
-  float o[2][4][4];
+  float o[GW][4][4];
 #pragma unroll
-  for (int gi = 0; gi < 2; ++gi)
+  for (int gi = 0; gi < GW; ++gi)
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -149,7 +156,7 @@ __global__ void __launch_bounds__(128, 4) attn_kernel(AttnArgs a) {
   for (int b = 0; b < nblk; ++b) {
     // refill the stage block b - 1 used (every warp finished it at the last barrier)
     const int nb = b + kAttnStages - 1;
-    if (nb < nblk) attn_issue(sm.st[nb % kAttnStages], a, rid, beg + nb * kAttnCells, end, kvh);
+    if (nb < nblk) attn_issue<NT>(sm.st[nb % kAttnStages], a, rid, beg + nb * kAttnCells, end, kvh);
     cp_async_commit();
     cp_async_wait<kAttnStages - 1>();
     __syncthreads();
@@ -163,8 +170,8 @@ __global__ void __launch_bounds__(128, 4) attn_kernel(AttnArgs a) {
       for (int c = 0; c < 4; ++c) s[nt][c] = 0.f;
       const int8_t* krow = st.k + (8 * nt + g) * kAttnKStride;
 #pragma unroll
-      for (int gi = 0; gi < 2; ++gi) {
-        const int qg = 2 * warp + gi;
+      for (int gi = 0; gi < GW; ++gi) {
+        const int qg = GW * warp + gi;
         const uint2 kw = *reinterpret_cast<const uint2*>(krow + 32 * qg + 8 * t);
         const uint32_t x0 = kw.x ^ 0x80808080u, x1 = kw.y ^ 0x80808080u;
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -186,7 +193,7 @@ __global__ void __launch_bounds__(128, 4) attn_kernel(AttnArgs a) {
     for (int nt = 0; nt < 4; ++nt) {
       float4 r = sm.red[0][nt][lane];
 #pragma unroll
-      for (int w = 1; w < 4; ++w) {
+      for (int w = 1; w < W; ++w) {
         const float4 y = sm.red[w][nt][lane];
         r.x += y.x;
         r.y += y.y;
@@ -230,7 +237,7 @@ __global__ void __launch_bounds__(128, 4) attn_kernel(AttnArgs a) {
       m_run[r] = mnew[r];
     }
 #pragma unroll
-    for (int gi = 0; gi < 2; ++gi)
+    for (int gi = 0; gi < GW; ++gi)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         o[gi][i][0] *= alpha[0];
@@ -249,8 +256,8 @@ __global__ void __launch_bounds__(128, 4) attn_kernel(AttnArgs a) {
       pa[3] = pack_half2(s[2 * s2 + 1][2], s[2 * s2 + 1][3]);
       const int cA = 16 * s2 + 2 * t;  // cells of k-index 2t, 2t+1, 2t+8, 2t+9
 #pragma unroll
-      for (int gi = 0; gi < 2; ++gi) {
-        const int qg = 2 * warp + gi;
+      for (int gi = 0; gi < GW; ++gi) {
+        const int qg = GW * warp + gi;
         // column g of n-tile i is dim 32qg + 4g + i
         const int8_t* vb = st.v + 32 * qg + 4 * g;
         const uint32_t wA = *reinterpret_cast<const uint32_t*>(vb + cA * kAttnVStride) ^ 0x80808080u;
@@ -284,8 +291,8 @@ __global__ void __launch_bounds__(128, 4) attn_kernel(AttnArgs a) {
     const int head = kvh * kQPerKV + hr;
     const size_t rh = static_cast<size_t>(row) * kHQ + head;
 #pragma unroll
-    for (int gi = 0; gi < 2; ++gi) {
-      const int dbase = 32 * (2 * warp + gi) + 8 * t;
+    for (int gi = 0; gi < GW; ++gi) {
+      const int dbase = 32 * (GW * warp + gi) + 8 * t;
       float4 lo = make_float4(o[gi][0][2 * r], o[gi][1][2 * r], o[gi][2][2 * r], o[gi][3][2 * r]);
       float4 hi = make_float4(o[gi][0][2 * r + 1], o[gi][1][2 * r + 1], o[gi][2][2 * r + 1],
                               o[gi][3][2 * r + 1]);
