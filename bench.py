@@ -39,7 +39,8 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 KERNEL_SOURCES = {
     "attn_kernel": "qsa_attn.cuh",
     "index_score_kernel": "qsa_index_score.cuh",
-    "topk_final_kernel": "qsa_topk.cuh",
+    "score_gemm_kernel": "qsa_score_gemm.cuh",
+    "topk": "qsa_topk_cluster.cuh",
     "merge_kernel": "qsa_merge.cuh",
 }
 CELL_BYTES = 2 * 2 * 256 + 2 * 2 * 8 * 2      # K + V codes and their scales, both KV heads
@@ -168,7 +169,7 @@ def source_hash(kernel: str) -> str:
 def traffic_for(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, or None if the
     kernel source changed since the counters were taken."""
-    if not os.path.exists(TRAFFIC_FILE):
+    if not os.path.exists(TRAFFIC_FILE) or kernel not in KERNEL_SOURCES:
         return None
     t = json.load(open(TRAFFIC_FILE)).get(workload, {}).get(kernel)
     if not t or t.get("source_sha") != source_hash(kernel):
@@ -496,40 +497,61 @@ def auto_nsplit(rows, top_k):
 
 
 def roofline(spec, kern, pk):
-    """Algorithmic bytes (or flops) per launch over measured launch time."""
-    info, avg, L = kern["info"], kern["avg_ms"], kern["launches"]
+    """Algorithmic bytes (or flops) per launch over measured launch time, for
+    every step kernel; the dominant one (most time per call) is `main`."""
+    info, avg = kern["info"], kern["avg_ms"]
     calls = len(spec.ns)
-    hbm = pk["hbm_gbs"]
+    hbm, tensor = pk["hbm_gbs"], pk["bf16_tflops"]
+    rows = info["rows"] / calls
+    ncells = info["ncells"] / calls                      # (row, cell) scores per call
     kernels = {}
-    # index score: every cell's key read once, every score written once
-    score_bytes = spec.L * KEY_BYTES * calls + 4 * info["ncells"]
-    kernels["index_score_kernel"] = {"ms": avg["index_score_kernel"], "bytes_per_launch": score_bytes / calls}
-    # attention: the union of the rows' selected cells (K, V, scales) + queries, ids, outputs
-    attn_bytes = info["union_cells"] * CELL_BYTES + info["rows"] * (24 * 256 * 4 * 2 + spec.top_k * 4)
-    kernels["attn_kernel"] = {"ms": avg["attn_kernel"], "bytes_per_launch": attn_bytes / calls}
-    kernels["topk"] = {"ms": avg["topk"]}
-    kernels["merge_kernel"] = {"ms": avg["merge_kernel"]}
-    out = {"kernels": kernels}
+
+    def hbm_entry(name, nbytes, note):
+        ms = avg[name]
+        if not ms:
+            return None
+        ach = nbytes / (ms / 1e3) / 1e9
+        return {"kernel": name, "bound": "hbm", "ms": ms, "bytes_per_launch": nbytes, "achieved": ach,
+                "peak": hbm, "unit": "GB/s", "frac": ach / hbm, "note": note}
+
+    # index score: keys once, scores written once (decode); prefill: 512 flops per visible cell
+    key_bytes = spec.L * KEY_BYTES
     if spec.kind == "decode":
-        dom = max(["index_score_kernel", "attn_kernel"], key=lambda k: avg[k] or 0)
-        b = kernels[dom]["bytes_per_launch"]
-        achieved = b / (avg[dom] / 1e3) / 1e9
-        out["main"] = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                       "frac": achieved / hbm, "peak_source": pk["source"],
-                       "traffic": traffic_for(dom, spec.name)}
-        both_b = (score_bytes - 4 * info["ncells"]) / calls + attn_bytes / calls
+        kernels["index_score_kernel"] = hbm_entry("index_score_kernel", key_bytes + 4 * ncells,
+                                                  "keys read once + fp32 scores written")
+    else:
+        ms = avg["index_score_kernel"]
+        flops = 512.0 * info["cells_scored"] / calls
+        ach = flops / (ms / 1e3) / 1e12
+        kernels["index_score_kernel"] = {"kernel": "score_gemm_kernel (tcgen05)", "bound": "tensor", "ms": ms,
+                                         "flops_per_launch": flops, "achieved": ach, "peak": tensor,
+                                         "unit": "TFLOP/s", "frac": ach / tensor,
+                                         "note": "512 flops per visible (row, cell); fp16 has bf16's nominal rate"}
+    # selection: every visible score read, ids written
+    kernels["topk"] = hbm_entry("topk", 4 * info["cells_scored"] / calls + 4 * rows * spec.top_k,
+                                "visible scores read + ids written (decode: one cluster kernel; "
+                                "prefill: histogram, filter and final kernels together)")
+    # attention: the union of the rows' selected cells (K, V, scales) + queries, ids, outputs
+    attn_bytes = (info["union_cells"] * CELL_BYTES + info["rows"] * (24 * 256 * 4 * 2 + spec.top_k * 4)) / calls
+    kernels["attn_kernel"] = hbm_entry("attn_kernel", attn_bytes,
+                                       "union of the rows' selected cells x 1088 B + q, ids, out"
+                                       + (" (prefill: gathered from L2 mostly)" if spec.kind == "prefill" else ""))
+    if avg["merge_kernel"]:
+        ns = info["nsplit"]
+        part_bytes = sum(n * 24 * ns[n] * 258 * 4 + n * 24 * 256 * 4 for n in ns) / calls
+        kernels["merge_kernel"] = hbm_entry("merge_kernel", part_bytes, "partials read + output written")
+    kernels = {k: v for k, v in kernels.items() if v}
+    dom = max(kernels, key=lambda k: kernels[k]["ms"] or 0)
+    main = dict(kernels[dom])
+    main["peak_source"] = pk["source"]
+    main["traffic"] = traffic_for(dom, spec.name)
+    out = {"kernels": kernels, "main": main}
+    if spec.kind == "decode":
+        both_b = key_bytes + attn_bytes
         both_t = (avg["index_score_kernel"] + avg["attn_kernel"]) / 1e3
         out["score_attn"] = {"bound": "hbm", "achieved": both_b / both_t / 1e9, "peak": hbm, "unit": "GB/s",
                              "frac": both_b / both_t / 1e9 / hbm,
                              "note": "keys + union of selected cells over the two kernels' summed time"}
-    else:
-        flops = 512.0 * info["cells_scored"] / calls
-        achieved = flops / (avg["index_score_kernel"] / 1e3) / 1e12
-        peak = pk["bf16_tflops"]
-        out["main"] = {"kernel": "index_score_kernel", "bound": "tensor", "achieved": achieved,
-                       "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                       "peak_source": pk["source"] + " bf16 dense (fp16 nominal ratio 1.0)",
-                       "traffic": traffic_for("index_score_kernel", spec.name)}
     return out
 
 
