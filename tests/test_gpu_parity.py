@@ -261,6 +261,55 @@ def test_attn_vs_oracle(gpu, nsplit, rows):
             assert rel_err(po[full] / pl[full][:, None], o[full] / l[full][:, None]) <= OUT_TOL
 
 
+def _check_attn(qsa, cache_h, cache, q, ids, nsplit, scale=1 / 16):
+    res = qsa.attn(cache, torch.from_numpy(q).to(DEV), torch.from_numpy(ids).to(DEV), nsplit, scale)
+    out = (res if nsplit == 1 else qsa.merge(res)).cpu().numpy()
+    for r in range(q.shape[0]):
+        assert rel_err(out[r], oracle.attn_row(cache_h, q[r], ids[r], scale)) <= OUT_TOL, f"row {r}"
+    return res
+
+
+# more than 8 rows (the prompt-chunk kernel): ragged last blocks, rows with one or
+# no cell, splits past the end of the list
+@pytest.mark.parametrize("rows,k,nsplit", [(9, 200, 1), (16, 129, 1), (10, 100, 64), (33, 2048, 3)])
+def test_attn_many_rows_shapes(gpu, rows, k, nsplit):
+    qsa = gpu
+    cells = 4096
+    wl = synth.make_workload(0, cells=cells)
+    q, _, _ = synth.make_queries(211, rows)
+    nvalid = [k, 1, 0] + [(k * (r + 1)) // rows for r in range(rows - 3)]
+    ids = _id_lists(212, rows, cells, k, nvalid)
+    cache = qsa.DeviceCache.from_host(wl.cache, DEV)
+    res = _check_attn(qsa, wl.cache, cache, q, ids, nsplit)
+    if nsplit > 1:
+        part = res.cpu().numpy()
+        empty = part[:, :, :, 1] == 0
+        assert np.all(np.isneginf(part[:, :, :, 0][empty])) and np.all(part[:, :, :, 2:][empty] == 0)
+        assert np.all(empty[2])  # the row without cells
+
+
+def test_attn_rising_maxima(gpu):
+    """Cells listed by ascending logit, so the running maximum keeps moving (by more
+    than 2^8 between the first and the last 128 cells) and the accumulated output
+    is rescaled many times."""
+    qsa = gpu
+    rows, cells, k = 9, 4096, 1024
+    cache_h = synth.make_cache(214, cells)
+    q, _, _ = synth.make_queries(215, rows)
+    q *= 2
+    kd = cache_h.k.astype(np.float64) * np.repeat(cache_h.ks.astype(np.float64), 32, -1)
+    ids = np.empty((rows, k), np.int32)
+    for r in range(rows):
+        logit = kd[:, 0, :] @ q[r, r % 12].astype(np.float64) / 16
+        order = np.argsort(logit, kind="stable")
+        ids[r] = order[::cells // k][:k]
+        # log2-domain maxima of the 128-cell tiles: the last one is far above the first
+        tmax = (logit[ids[r]] / np.log(2)).reshape(-1, 128).max(1)
+        assert tmax[-1] - tmax[0] > 8 + 1
+    _check_attn(qsa, cache_h, qsa.DeviceCache.from_host(cache_h, DEV), q, ids, 1)
+    _check_attn(qsa, cache_h, qsa.DeviceCache.from_host(cache_h, DEV), q, ids, 5)
+
+
 def test_attn_small_v_scales(gpu):
     qsa = gpu
     cells = 2000

@@ -25,9 +25,7 @@
 //     in-flight copies and MMAs are drained (again with a bound) and TMEM is freed.
 #pragma once
 
-#include <cuda.h>
-
-#include "qsa_common.cuh"
+#include "qsa_sm100.cuh"
 
 namespace qsa {
 
@@ -46,8 +44,6 @@ constexpr int kGemmSmemBytes = kGemmABytes + kGemmStages * kGemmBBytes + 4 * kGe
 // TMEM (the CTA allocates all 512 columns).
 constexpr int kGemmSmemRequest = kGemmSmemBytes;
 static_assert(kGemmSmemRequest > 114 * 1024, "one GEMM CTA per SM");
-constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // one second
-constexpr uint32_t kStatusTimeout = 4;                       // QSA_ERR_TIMEOUT
 
 struct GemmArgs {
   const float* iw;     // [T][4]
@@ -72,140 +68,11 @@ struct __align__(8) GemmBarriers {
   uint32_t abort;
 };
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count));
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ unsigned long long global_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
-  return t;
-}
-
-// Wait for the phase of `bar` with parity `parity`.  Returns false if the CTA
-// is aborting or the wait exceeded its limit (which starts the abort).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, GemmBarriers& gb,
-                                          uint32_t* status) {
-  const uint32_t addr = smem_u32(bar);
-  unsigned long long t0 = 0;
-  for (uint32_t it = 0;; ++it) {
-    uint32_t done;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(done)
-        : "r"(addr), "r"(parity)
-        : "memory");
-    if (done) return true;
-    if (*reinterpret_cast<volatile uint32_t*>(&gb.abort)) return false;
-    if ((it & 255u) == 0u) {
-      const unsigned long long now = global_ns();
-      if (t0 == 0) t0 = now;
-      else if (now - t0 > kWaitLimitNs) {
-        atomicExch(status, kStatusTimeout);
-        *reinterpret_cast<volatile uint32_t*>(&gb.abort) = 1u;
-        return false;
-      }
-    }
-  }
-}
-
-// Wait with a bound but never start an abort (used while draining).
-__device__ __forceinline__ void mbar_drain_wait(uint64_t* bar, uint32_t parity) {
-  const uint32_t addr = smem_u32(bar);
-  const unsigned long long t0 = global_ns();
-  for (;;) {
-    uint32_t done;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(done)
-        : "r"(addr), "r"(parity)
-        : "memory");
-    if (done || global_ns() - t0 > kWaitLimitNs) return;
-  }
-}
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(
-          smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(
-          smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int x, int y, const void* src) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];\n" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(x), "r"(y), "r"(smem_u32(src))
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void bulk_wait_read() {
-  asm volatile("cp.async.bulk.wait_group.read %0;\n" ::"n"(N) : "memory");
-}
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-}
-
-// UMMA shared-memory descriptor: K-major operand rows of 128 bytes with the
-// 128-byte swizzle (8-row atoms of 1024 bytes: leading offset 16 B, stride 1024 B).
-__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
-  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (1ull << 16) | (64ull << 32) | (1ull << 46) |
-         (2ull << 61);
-}
-
 // Instruction descriptor: fp32 accumulate, fp16 A and B, both K-major, M = 128, N = 64.
-constexpr uint32_t kGemmIdesc = (1u << 4) | (static_cast<uint32_t>(kGemmCells >> 3) << 17) |
-                                (static_cast<uint32_t>(kGemmTokens >> 4) << 24);
+constexpr uint32_t kGemmIdesc = umma_idesc_f16(kGemmTokens, kGemmCells, false, false);
 
-__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(kGemmIdesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
-                   smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
+// A K-major operand here is a stack of 8-row atoms of 1024 bytes.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) { return umma_desc_k_sw128(saddr, 1024); }
 
 // grid: number of SMs (persistent); block: kGemmThreads; dynamic smem: kGemmSmemRequest.
 __global__ void __launch_bounds__(kGemmThreads, 1)
@@ -243,13 +110,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     mbar_init(&gb.drain, 1);
     gb.abort = 0u;
-    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    mbar_init_fence();
   }
-  if (warp == 1) {  // allocate all 512 TMEM columns (two accumulators of 4 heads x 64)
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(&gb.tmem_base)),
-                 "r"(512u));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::);
-  }
+  if (warp == 1) tmem_alloc(&gb.tmem_base, 512u);  // two accumulators of 4 heads x 64 columns
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -265,7 +128,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int it = it0; it < it1 && ok; ++it) {
         const int tb = it / nct, ct = it % nct;
         if (tb != cur_tb) {
-          if (a_loads > 0) ok = mbar_wait(&gb.a_empty, (a_loads - 1) & 1, gb, a.status);
+          if (a_loads > 0) ok = mbar_wait(&gb.a_empty, (a_loads - 1) & 1, &gb.abort, a.status);
           if (!ok) break;
           mbar_expect_tx(&gb.a_full, kGemmABytes);
           for (int h = 0; h < kHI; ++h)
@@ -274,7 +137,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           ++a_loads;
         }
         const int li = it - it0, s = li % kGemmStages, round = li / kGemmStages;
-        ok = mbar_wait(&gb.b_empty[s], (round & 1) ^ 1, gb, a.status);
+        ok = mbar_wait(&gb.b_empty[s], (round & 1) ^ 1, &gb.abort, a.status);
         if (!ok) break;
         mbar_expect_tx(&gb.b_full[s], kGemmBBytes);
         tma_load_2d(sB + s * kGemmBBytes, &tmap_key, 0, ct * kGemmCells, &gb.b_full[s]);
@@ -297,13 +160,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int li = it - it0, s = li % kGemmStages, round = li / kGemmStages;
         const int buf = li & 1, bround = li >> 1;
         if (tb != cur_tb) {
-          ok = mbar_wait(&gb.a_full, a_loads & 1, gb, a.status);
+          ok = mbar_wait(&gb.a_full, a_loads & 1, &gb.abort, a.status);
           if (!ok) break;
           cur_tb = tb;
           ++a_loads;
         }
-        ok = mbar_wait(&gb.b_full[s], round & 1, gb, a.status) &&
-             mbar_wait(&gb.acc_empty[buf], (bround & 1) ^ 1, gb, a.status);
+        ok = mbar_wait(&gb.b_full[s], round & 1, &gb.abort, a.status) &&
+             mbar_wait(&gb.acc_empty[buf], (bround & 1) ^ 1, &gb.abort, a.status);
         if (!ok) break;
         tc_fence_after();
         const uint32_t b0 = smem_u32(sB + s * kGemmBBytes);
@@ -313,7 +176,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t d = tmem + static_cast<uint32_t>(buf * 256 + h * kGemmCells);
 #pragma unroll
           for (int ks = 0; ks < kDI / 16; ++ks)
-            umma_f16(d, umma_desc_sw128(a0 + ks * 32), umma_desc_sw128(b0 + ks * 32), ks > 0 ? 1u : 0u);
+            umma_f16(d, umma_desc_sw128(a0 + ks * 32), umma_desc_sw128(b0 + ks * 32), kGemmIdesc, ks > 0 ? 1u : 0u);
         }
         umma_commit(&gb.b_empty[s]);       // the key stage is free once these MMAs finish
         umma_commit(&gb.acc_full[buf]);    // the accumulator is ready for the epilogue
@@ -331,7 +194,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int it = it0; it < it1; ++it) {
         const int tb = it / nct, ct = it % nct;
         const int li = it - it0, sb = li & 1;
-        if (!mbar_wait(&gb.stage_full[sb], (li >> 1) & 1, gb, a.status)) break;
+        if (!mbar_wait(&gb.stage_full[sb], (li >> 1) & 1, &gb.abort, a.status)) break;
         for (int h = 0; h < 2; ++h)  // a box past the last column has nothing to write
           if (ct * kGemmCells + 32 * h < a.ncells)
             tma_store_2d(&tmap_out, ct * kGemmCells + 32 * h, tb * kGemmTokens,
@@ -361,12 +224,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         cur_tb = tb;
       }
       // one lane waits, the warp follows it (the TMEM loads below are warp-collective)
-      uint32_t ok = 1u;
-      if (lane == 0) ok = mbar_wait(&gb.acc_full[buf], bround & 1, gb, a.status) ? 1u : 0u;
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      __syncwarp();
+      if (!mbar_wait_warp(&gb.acc_full[buf], bround & 1, &gb.abort, a.status)) break;
       tc_fence_after();
-      if (!ok) break;
       const int col = colq * 16;
       uint32_t rr[kHI][16];
 #pragma unroll
@@ -390,10 +249,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // stage the scores: buffer li & 1, half colq / 2, 128-byte rows with 16-byte
       // chunk c stored at c ^ (row % 8) (the layout the TMA store's 128-byte swizzle reads)
       const int sb = li & 1;
-      ok = 1u;
-      if (lane == 0) ok = mbar_wait(&gb.stage_free[sb], ((li >> 1) & 1) ^ 1, gb, a.status) ? 1u : 0u;
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
+      if (!mbar_wait_warp(&gb.stage_free[sb], ((li >> 1) & 1) ^ 1, &gb.abort, a.status)) break;
       unsigned char* half = sC + (sb * 2 + (colq >> 1)) * kGemmCHalfBytes + r * 128;
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
@@ -410,7 +266,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(512u));
+  if (warp == 1) tmem_dealloc(tmem, 512u);
 }
 
 // Self-test of the bounded wait: one thread waits on a barrier that nothing
@@ -420,8 +276,8 @@ __global__ void wait_selftest_kernel(uint32_t* status) {
   if (threadIdx.x == 0) {
     mbar_init(&gb.drain, 1);
     gb.abort = 0u;
-    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-    mbar_wait(&gb.drain, 0, gb, status);
+    mbar_init_fence();
+    mbar_wait(&gb.drain, 0, &gb.abort, status);
   }
 }
 
