@@ -16,7 +16,10 @@
 //    online softmax and accumulates P.V for its own 128 dims;
 //  * int8 codes become fp16 exactly (byte-permute with the 0x6400 exponent).  The
 //    per-32 K scale multiplies each 32-dim partial product in fp32 after the
-//    MMA; the per-32 V scale multiplies the fp16 V operand.  Q and P are fp16.
+//    MMA; the per-32 V scale multiplies the fp16 V operand.  Q and P are fp16;
+//  * the reference maximum of the online softmax moves only when a block
+//    exceeds it by more than 2^8, so P stays <= 256 and most blocks skip the
+//    rescale of O; split partials are reported against the true maximum.
 #pragma once
 
 #include "qsa_common.cuh"
@@ -36,6 +39,8 @@ struct __align__(16) AttnStage {
 };
 
 constexpr int kAttnStages = 2;
+constexpr float kAttnShift = 8.f;      // log2 margin before the reference maximum moves
+constexpr float kAttnNoMax = -1.0e30f;  // reference maximum before the first valid cell
 
 // W warps split the 256 dims (W = 4 for the latency of decode, 2 for the
 // throughput of prefill: half the duplicated softmax and score-reduction work).
@@ -143,7 +148,10 @@ __global__ void __launch_bounds__(32 * W) attn_kernel(AttnArgs a) {
     cp_async_commit();
   }
 
-  float m_run[2] = {-INFINITY, -INFINITY};
+  // reference maximum (log2 units) of P: finite from the start, so a block with
+  // no valid cell gives exp2(-inf - m_run) = 0 without a guard
+  float m_run[2] = {kAttnNoMax, kAttnNoMax};
+  float m_top[2] = {-INFINITY, -INFINITY};  // true maximum
   float l_run[2] = {0.f, 0.f};
   float o[GW][4][4];
 #pragma unroll
@@ -161,6 +169,7 @@ __global__ void __launch_bounds__(32 * W) attn_kernel(AttnArgs a) {
     cp_async_wait<kAttnStages - 1>();
     __syncthreads();
     const AttnStage& st = sm.st[b % kAttnStages];
+    const uint32_t valid = __ballot_sync(0xffffffffu, st.valid[lane] != 0);  // bit c: slot c holds a cell
 
     // ---- partial scores over this warp's 64 dims
     float s[4][4];
@@ -177,12 +186,12 @@ __global__ void __launch_bounds__(32 * W) attn_kernel(AttnArgs a) {
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
         mma_f16_16816(acc, aq[gi][0], i8x2_to_h2(x0, 0x4140u), i8x2_to_h2(x0, 0x4342u));
         mma_f16_16816(acc, aq[gi][1], i8x2_to_h2(x1, 0x4140u), i8x2_to_h2(x1, 0x4342u));
-        const float sc0 = __half2float(st.ks[(8 * nt + 2 * t) * kNG + qg]);
-        const float sc1 = __half2float(st.ks[(8 * nt + 2 * t + 1) * kNG + qg]);
-        s[nt][0] = fmaf(sc0, acc[0], s[nt][0]);
-        s[nt][1] = fmaf(sc1, acc[1], s[nt][1]);
-        s[nt][2] = fmaf(sc0, acc[2], s[nt][2]);
-        s[nt][3] = fmaf(sc1, acc[3], s[nt][3]);
+        const float2 sc = make_float2(__half2float(st.ks[(8 * nt + 2 * t) * kNG + qg]),
+                                      __half2float(st.ks[(8 * nt + 2 * t + 1) * kNG + qg]));
+        s[nt][0] = fmaf(sc.x, acc[0], s[nt][0]);
+        s[nt][1] = fmaf(sc.y, acc[1], s[nt][1]);
+        s[nt][2] = fmaf(sc.x, acc[2], s[nt][2]);
+        s[nt][3] = fmaf(sc.y, acc[3], s[nt][3]);
       }
       sm.red[warp][nt][lane] = make_float4(s[nt][0], s[nt][1], s[nt][2], s[nt][3]);
     }
@@ -191,16 +200,22 @@ __global__ void __launch_bounds__(32 * W) attn_kernel(AttnArgs a) {
     float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt) {
-      float4 r = sm.red[0][nt][lane];
+      float4 r;
+      if constexpr (W == 2) {  // own partial + the other warp's (a + b == b + a: both warps agree)
+        const float4 y = sm.red[warp ^ 1][nt][lane];
+        r = make_float4(s[nt][0] + y.x, s[nt][1] + y.y, s[nt][2] + y.z, s[nt][3] + y.w);
+      } else {
+        r = sm.red[0][nt][lane];
 #pragma unroll
-      for (int w = 1; w < W; ++w) {
-        const float4 y = sm.red[w][nt][lane];
-        r.x += y.x;
-        r.y += y.y;
-        r.z += y.z;
-        r.w += y.w;
+        for (int w = 1; w < W; ++w) {
+          const float4 y = sm.red[w][nt][lane];
+          r.x += y.x;
+          r.y += y.y;
+          r.z += y.z;
+          r.w += y.w;
+        }
       }
-      const bool v0 = st.valid[8 * nt + 2 * t], v1 = st.valid[8 * nt + 2 * t + 1];
+      const bool v0 = (valid >> (8 * nt + 2 * t)) & 1u, v1 = (valid >> (8 * nt + 2 * t + 1)) & 1u;
       s[nt][0] = v0 ? r.x : -INFINITY;
       s[nt][1] = v1 ? r.y : -INFINITY;
       s[nt][2] = v0 ? r.z : -INFINITY;
@@ -213,11 +228,26 @@ __global__ void __launch_bounds__(32 * W) attn_kernel(AttnArgs a) {
       mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
       mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
     }
-    float alpha[2], mnew[2];
+    // The reference maximum m_run moves only when a block exceeds it by more
+    // than 2^8 (P <= 256 in fp16), so most blocks skip the rescale of O; the
+    // true maximum m_top is kept for the split partials.
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      mnew[r] = fmaxf(m_run[r], mx[r]);
-      alpha[r] = (mnew[r] == -INFINITY) ? 1.f : exp2f(m_run[r] - mnew[r]);
+    for (int r = 0; r < 2; ++r) m_top[r] = fmaxf(m_top[r], mx[r]);
+    if (__any_sync(0xffffffffu, mx[0] > m_run[0] + kAttnShift || mx[1] > m_run[1] + kAttnShift)) {
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const float mnew = fmaxf(m_run[r], mx[r]);
+        const float alpha = exp2f(m_run[r] - mnew);
+        l_run[r] *= alpha;
+        m_run[r] = mnew;
+#pragma unroll
+        for (int gi = 0; gi < GW; ++gi)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            o[gi][i][2 * r] *= alpha;
+            o[gi][i][2 * r + 1] *= alpha;
+          }
+      }
     }
     float rs[2] = {0.f, 0.f};
 #pragma unroll
@@ -225,7 +255,7 @@ __global__ void __launch_bounds__(32 * W) attn_kernel(AttnArgs a) {
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int r = c >> 1;
-        const float p = (mnew[r] == -INFINITY) ? 0.f : exp2f(s[nt][c] - mnew[r]);
+        const float p = exp2f(s[nt][c] - m_run[r]);
         s[nt][c] = p;
         rs[r] += p;
       }
@@ -233,18 +263,8 @@ __global__ void __launch_bounds__(32 * W) attn_kernel(AttnArgs a) {
     for (int r = 0; r < 2; ++r) {
       rs[r] += __shfl_xor_sync(0xffffffffu, rs[r], 1);
       rs[r] += __shfl_xor_sync(0xffffffffu, rs[r], 2);
-      l_run[r] = l_run[r] * alpha[r] + rs[r];
-      m_run[r] = mnew[r];
+      l_run[r] += rs[r];
     }
-#pragma unroll
-    for (int gi = 0; gi < GW; ++gi)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        o[gi][i][0] *= alpha[0];
-        o[gi][i][1] *= alpha[0];
-        o[gi][i][2] *= alpha[1];
-        o[gi][i][3] *= alpha[1];
-      }
 
     // ---- P.V for this warp's 64 dims; P's k-index j <-> cell 16*s2 + j
 #pragma unroll
@@ -303,15 +323,18 @@ __global__ void __launch_bounds__(32 * W) attn_kernel(AttnArgs a) {
         float* dst = a.out + rh * kD + dbase;
         *reinterpret_cast<float4*>(dst) = lo;
         *reinterpret_cast<float4*>(dst + 4) = hi;
-      } else {
+      } else {  // partials relative to the true maximum
+        const float corr = (m_top[r] == -INFINITY) ? 0.f : exp2f(m_run[r] - m_top[r]);
+        lo.x *= corr; lo.y *= corr; lo.z *= corr; lo.w *= corr;
+        hi.x *= corr; hi.y *= corr; hi.z *= corr; hi.w *= corr;
         float* dst = a.part + (rh * a.nsplit + split) * kPart;
         *reinterpret_cast<float2*>(dst + 2 + dbase) = make_float2(lo.x, lo.y);
         *reinterpret_cast<float2*>(dst + 2 + dbase + 2) = make_float2(lo.z, lo.w);
         *reinterpret_cast<float2*>(dst + 2 + dbase + 4) = make_float2(hi.x, hi.y);
         *reinterpret_cast<float2*>(dst + 2 + dbase + 6) = make_float2(hi.z, hi.w);
         if (warp == 0 && t == 0) {
-          dst[0] = m_run[r] == -INFINITY ? -INFINITY : m_run[r] * kLn2;
-          dst[1] = l_run[r];
+          dst[0] = m_top[r] == -INFINITY ? -INFINITY : m_top[r] * kLn2;
+          dst[1] = l_run[r] * corr;
         }
       }
     }
