@@ -491,8 +491,8 @@ def kernel_times(qsa, torch, spec, caches, wl, q, iq, iw, ws, dev, stream, reps)
 
 
 def auto_nsplit(rows, top_k):
-    """The library's automatic split count (qsa_api.cu): one wave of 4 CTAs per SM."""
-    want = (4 * 148) // (2 * rows)
+    """The library's automatic split count (qsa_api.cu): about 256 CTAs in all."""
+    want = 128 // rows
     return max(1, min(64, max(1, top_k // 32), want))
 
 

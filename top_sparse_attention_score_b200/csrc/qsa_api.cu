@@ -182,9 +182,11 @@ struct StepPlan {
 };
 
 int auto_nsplit(int rows, int top_k) {
-  // As many (row, KV head, split) CTAs as one wave holds (4 per SM on 148 SMs),
-  // pieces of at least 32 cells; large prefill chunks need no splits.
-  const int want = (4 * 148) / (2 * rows);
+  // About 256 (row, KV head, split) CTAs, pieces of at least 32 cells: on a B200
+  // the attention plus the merge of a decode step of 1-8 rows is fastest there
+  // (more splits shorten the gathers but lengthen the merge); large prefill
+  // chunks need no splits.
+  const int want = 128 / rows;
   return std::max(1, std::min({QSA_MAX_SPLITS, std::max(1, top_k / 32), want}));
 }
 
