@@ -183,7 +183,7 @@ def make_new_cells(seed: int, n: int):
 
 # The five workloads: decode at 4K/64K/256K cells, prefill chunks at 64K/256K.
 CONFIGS = {
-    0: dict(kind="decode", L=4096, n=1, top_k=512, nsplit=1),
+    0: dict(kind="decode", L=4096, n=1, top_k=512, nsplit=0),
     1: dict(kind="decode", L=65536, n=8, top_k=2048, nsplit=0, outlier_frac=0.01),
     2: dict(kind="decode", L=262144, n=1, top_k=2048, nsplit=64, outlier_frac=0.01),
     3: dict(kind="prefill", L=65536, T=2048, pos0=63488, top_k=2048, nsplit=1),
