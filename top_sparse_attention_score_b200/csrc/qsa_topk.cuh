@@ -31,9 +31,8 @@ constexpr int kMaxWindowBits = 1 << 18;  // cells per bitmap window (two 32 KB b
 
 // Per-row counters, zeroed before every use.
 enum : int {
-  kCtrSure = 0, kCtrCand = 1, kCtrHistDone = 2, kCtrSelectDone = 3, kCtrThrBin = 4,
-  kCtrAbove = 5, kCtrAttnDone = 6,  // + KV head (6, 7)
-  kCtrWords = 8
+  kCtrSure = 0, kCtrCand = 1, kCtrHistDone = 2, kCtrThrBin = 4, kCtrAbove = 5,
+  kCtrWords = 8  // words 3, 6 and 7 are spare (the layout and its size stay fixed)
 };
 
 struct TopkWs {
