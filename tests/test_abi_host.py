@@ -104,3 +104,16 @@ def test_prefill_and_steps_reject_bad_arguments(lib):
     assert lib.qsa_attn(cb, 1, P, P, 64, 1, 0.0625, P, None, None) == 1  # nsplit 1 needs out
     assert lib.qsa_merge(None, 1, 2, P, None) == 1
     assert lib.qsa_merge(P, 1, 65, P, None) == 1
+
+
+def test_bench_split_rule_matches_the_library(lib):
+    """bench.py reports the split count the library picks for nsplit = 0; the
+    workspace holds the split partials, so its size shows which count was used."""
+    import bench
+    for n in range(1, 9):
+        for k in (512, 2048):
+            auto = lib.qsa_workspace_bytes(0, n, 65536, k, 0)
+            assert auto == lib.qsa_workspace_bytes(0, n, 65536, k, bench.auto_nsplit(n, k)), (n, k)
+            other = bench.auto_nsplit(n, k) + 1
+            if other <= 64:
+                assert auto != lib.qsa_workspace_bytes(0, n, 65536, k, other), (n, k)
