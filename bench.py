@@ -179,7 +179,9 @@ def traffic_for(kernel: str, workload: str):
 
 # ---------------------------------------------------------------- distributed plumbing
 
-def dist_init(n):
+def dist_init(n, backend: str = "nccl"):
+    """Join the job's process group (one process per GPU; rendezvous from the
+    torchrun environment).  Returns (rank, world, local rank); (0, 1, 0) alone."""
     if n <= 1 or "RANK" not in os.environ:
         return 0, 1, 0
     import datetime
@@ -187,18 +189,23 @@ def dist_init(n):
     import torch
     import torch.distributed as dist
     local = int(os.environ.get("LOCAL_RANK", 0))
-    torch.cuda.set_device(local)
-    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                            device_id=torch.device("cuda", local))
+    if backend == "nccl":
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return dist.get_rank(), dist.get_world_size(), local
 
 
 def dist_max(x: float, world: int) -> float:
+    """The largest x over ranks (every rank calls it, in the same order)."""
     if world <= 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -207,6 +214,14 @@ def barrier(world: int):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
+
+
+def job_rate(units_per_step: float, steps: int, ms_local: float, world: int):
+    """Whole-job throughput of `world` replicas that each ran `steps` steps of
+    `units_per_step` units: all ranks' units over the slowest rank's time.
+    Returns (units per second, the slowest rank's milliseconds)."""
+    ms_max = dist_max(ms_local, world)
+    return world * units_per_step * steps / (ms_max / 1000.0), ms_max
 
 
 # ---------------------------------------------------------------- CPU oracle leg
@@ -354,8 +369,7 @@ def run_cuda(args, spec: Spec):
     launches = per_graph * steps
     ms = ev0.elapsed_time(ev1)
     barrier(world)
-    ms_max = dist_max(ms, world)
-    value = world * spec.units * steps / (ms_max / 1000.0)
+    value, ms_max = job_rate(spec.units, steps, ms, world)
 
     # ---- end to end through the public API from pinned host buffers
     q_h = torch.from_numpy(wl.q).pin_memory()
@@ -396,8 +410,7 @@ def run_cuda(args, spec: Spec):
         e2e_step(i)
     ev1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = dist_max(ev0.elapsed_time(ev1), world)
-    e2e_value = world * spec.units * steps / (e2e_ms / 1000.0)
+    e2e_value, _ = job_rate(spec.units, steps, ev0.elapsed_time(ev1), world)
 
     # ---- per-kernel durations, step-level calls with events on the same stream
     kern = kernel_times(qsa, torch, spec, caches, wl, q, iq, iw, ws, dev, stream, 20)
