@@ -204,6 +204,23 @@ def test_topk_candidate_overflow(gpu):
     _topk_case(gpu, s, V, 2048)
 
 
+def test_topk_threshold_bin_sizes(gpu):
+    # one row per size of the threshold bin, around the limits of the one-warp
+    # searches (in registers up to 1024 candidates, shared-memory digits beyond):
+    # 1800 cells clearly above, the bin's cells in [10.01, 10.4] (one fp16 bin) with
+    # 40 distinct values, so ties cross the CTAs' ranges, the rest far below
+    st = synth.Stream(108, "tk")
+    V, above, k = 60000, 1800, 2048
+    sizes = [250, 512, 513, 1024, 1025, 3000]
+    s = np.zeros((len(sizes), V + len(sizes)), np.float32)
+    for r, nb in enumerate(sizes):
+        s[r] = st.uniform(V + len(sizes), 0.0, 5.0)
+        pick = np.argsort(st.uniform(V), kind="stable")[:above + nb]
+        s[r, pick[:above]] = st.uniform(above, 20.0, 30.0)
+        s[r, pick[above:]] = 10.01 + np.floor(st.uniform(nb) * 40) * 0.01
+    _topk_case(gpu, s, V, k)
+
+
 def test_topk_many_windows(gpu):
     st = synth.Stream(106, "tk")
     V = (1 << 19) * 2 + 777

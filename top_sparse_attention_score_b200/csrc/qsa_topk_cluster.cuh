@@ -14,8 +14,10 @@
 //     shared memory and finds the threshold bin itself;
 //   * each CTA lists its cells in the threshold bin (typically a few hundred in
 //     the row); after a second barrier every CTA gathers all lists and one warp
-//     radix-selects the exact k-th key over the bits the candidates do not share,
-//     and derives every CTA's output offset from the gathered lists;
+//     finds the exact k-th key over the bits the candidates do not share: up to
+//     1024 candidates held in registers, one bit per step, otherwise 8-bit digits
+//     counted in shared memory; it derives every CTA's output offset from the
+//     gathered lists;
 //   * each CTA marks its selected cells (and the lowest-index ties) in a bitmap of
 //     its own contiguous range and writes them in ascending order.  A split
 //     arrive/wait cluster barrier keeps every CTA's shared memory alive until the
@@ -79,6 +81,101 @@ __device__ __forceinline__ void warp_threshold_256(const uint32_t* h, uint32_t k
   }
   bin = __shfl_sync(0xffffffffu, b, f);
   above = __shfl_sync(0xffffffffu, ab, f);
+}
+
+constexpr int kWarpSelSlots = 32;  // candidates per lane the register select holds (n <= 1024)
+
+// One warp: the need-th largest of the n gathered candidate keys (1 <= need <= n
+// <= 32 * S), decided one bit at a time from the highest bit the keys do not all
+// share.  Lane l holds candidates l, l + 32, ... in S registers, the empty slots
+// key 0; every step runs straight-line over all S slots (a branch per slot costs
+// more than its compare) and subtracts the empty slots' matches in one go.  The
+// search ends early once a single candidate is left on the prefix: its key is
+// the answer.  Returns the key in `thr` and, in `take`, how many candidates
+// equal to it are kept (need minus the candidates above it).  The candidates of
+// CTA q are the gathered range [q_off[q], q_off[q + 1]); lanes q < kClusterCtas
+// set q_sel[q] = q_sure[q] + (those above thr) and q_eq[q] = (those equal to
+// thr) from per-slot ballot words staged in words[0, 64).
+template <int S>
+__device__ __forceinline__ void warp_select_regs(const uint32_t* gkey, const uint32_t* q_off, uint32_t n,
+                                                 uint32_t need, const uint32_t* q_sure, uint32_t* q_sel,
+                                                 uint32_t* q_eq, uint32_t* words, uint32_t& thr, uint32_t& take) {
+  constexpr uint32_t full = 0xffffffffu;
+  const uint32_t lane = threadIdx.x & 31u;
+  const uint32_t mine = n > lane ? (n - lane + 31u) >> 5 : 0u;  // slots holding a key in this lane
+  const uint32_t empty = S - mine;
+  uint32_t k[S];
+  uint32_t k_and = full, k_or = 0u;
+#pragma unroll
+  for (int j = 0; j < S; ++j) {
+    k[j] = static_cast<uint32_t>(j) < mine ? gkey[j * 32 + lane] : 0u;
+    k_and &= static_cast<uint32_t>(j) < mine ? k[j] : full;
+    k_or |= k[j];
+  }
+  k_and = __reduce_and_sync(full, k_and);
+  k_or = __reduce_or_sync(full, k_or);
+  uint32_t diff = k_and ^ k_or;  // bits on which the candidates differ
+  uint32_t pf = k_and, mk = ~diff, nd = need, alive = n;
+  while (diff) {
+    const uint32_t bit = 0x80000000u >> __clz(diff);
+    diff ^= bit;
+    mk |= bit;
+    const uint32_t want = pf | bit;
+    uint32_t c0 = 0u, c1 = 0u;
+#pragma unroll
+    for (int j = 0; j < S; j += 2) {
+      c0 += ((k[j] ^ want) & mk) == 0u ? 1u : 0u;
+      if (j + 1 < S) c1 += ((k[j + 1] ^ want) & mk) == 0u ? 1u : 0u;
+    }
+    const uint32_t c = __reduce_add_sync(full, c0 + c1 - ((want & mk) == 0u ? empty : 0u));
+    if (nd <= c) {  // the need-th largest has this bit set
+      pf = want;
+      alive = c;
+    } else {  // all c are above it
+      nd -= c;
+      alive -= c;
+    }
+    if (alive == 1u) {  // the one candidate left on the prefix is the answer
+      uint32_t key = 0u;
+      bool hit = false;
+#pragma unroll
+      for (int j = 0; j < S; ++j) {
+        const bool h = static_cast<uint32_t>(j) < mine && ((k[j] ^ pf) & mk) == 0u;
+        key = h ? k[j] : key;
+        hit = hit || h;
+      }
+      const uint32_t who = __ballot_sync(full, hit);
+      pf = __shfl_sync(full, key, __ffs(who) - 1);
+      break;
+    }
+  }
+  uint32_t w_gt = 0u, w_eq = 0u;  // lane j: the ballot words of slot j
+#pragma unroll
+  for (int j = 0; j < S; ++j) {
+    const uint32_t base = static_cast<uint32_t>(j) * 32u;
+    const uint32_t valid = n >= base + 32u ? full : (n > base ? (1u << (n - base)) - 1u : 0u);
+    const uint32_t g = __ballot_sync(full, k[j] > pf) & valid;
+    const uint32_t e = __ballot_sync(full, k[j] == pf) & valid;
+    w_gt = lane == static_cast<uint32_t>(j) ? g : w_gt;
+    w_eq = lane == static_cast<uint32_t>(j) ? e : w_eq;
+  }
+  words[lane] = w_gt;
+  words[32 + lane] = w_eq;
+  __syncwarp();
+  if (lane < static_cast<uint32_t>(kClusterCtas)) {
+    const uint32_t a = q_off[lane], b = lane + 1u < static_cast<uint32_t>(kClusterCtas) ? q_off[lane + 1] : n;
+    uint32_t cg = 0u, ce = 0u;
+    for (uint32_t w = a >> 5; a < b && w <= (b - 1u) >> 5; ++w) {
+      const uint32_t lo = max(a, w * 32u) - w * 32u, hi = min(b, w * 32u + 32u) - w * 32u;
+      const uint32_t m = (hi == 32u ? full : (1u << hi) - 1u) & ~((1u << lo) - 1u);
+      cg += __popc(words[w] & m);
+      ce += __popc(words[32 + w] & m);
+    }
+    q_sel[lane] = q_sure[lane] + cg;
+    q_eq[lane] = ce;
+  }
+  thr = pf;
+  take = nd;
 }
 
 __device__ __forceinline__ void cluster_arrive() {
@@ -262,7 +359,20 @@ __global__ void __launch_bounds__(kClusterThreads) cluster_select_kernel(const f
     }
     cluster_arrive();
     __syncthreads();
-    if (tid < 32) {
+    if (tid < 32 && total_cand <= 32u * kWarpSelSlots) {
+      uint32_t pf, nd;
+      if (total_cand <= 256u)
+        warp_select_regs<8>(sm.gkey, sm.q_off, total_cand, need, sm.q_sure, sm.q_sel, sm.q_eq, sm.tmp256, pf, nd);
+      else if (total_cand <= 512u)
+        warp_select_regs<16>(sm.gkey, sm.q_off, total_cand, need, sm.q_sure, sm.q_sel, sm.q_eq, sm.tmp256, pf, nd);
+      else
+        warp_select_regs<kWarpSelSlots>(sm.gkey, sm.q_off, total_cand, need, sm.q_sure, sm.q_sel, sm.q_eq,
+                                        sm.tmp256, pf, nd);
+      if (lane == 0) {
+        sm.misc[2] = pf;
+        sm.misc[3] = nd;
+      }
+    } else if (tid < 32) {
       // warp 0: exact threshold key over the bits the candidates do not all share
       uint32_t k_and = 0xffffffffu, k_or = 0u;
       for (uint32_t i = lane; i < total_cand; i += 32) {
