@@ -300,24 +300,33 @@ __global__ void __launch_bounds__(kClusterThreads) cluster_select_kernel(const f
                          above);
 
   // ---- count this CTA's cells above the threshold bin; list the ones in it
-  uint32_t my_sure = 0u;
+  // (straight-line: per-thread counts, a warp scan, one append per warp)
+  uint32_t my_sure = 0u, my_cand = 0u;
 #pragma unroll
   for (int e = 0; e < PER; ++e) {
-    const int li = e * NT + tid;
     const uint32_t b = QSA_BIN(e);
-    const bool valid = c0 + li < V;
+    const bool valid = c0 + e * NT + tid < V;
     my_sure += (valid && b > thr_bin) ? 1u : 0u;
-    const bool is_cand = valid && b == thr_bin;
-    const uint32_t m = __ballot_sync(0xffffffffu, is_cand);
-    if (!m) continue;
-    const int leader = __ffs(m) - 1;
+    my_cand += (valid && b == thr_bin) ? 1u : 0u;
+  }
+  {
+    uint32_t incl = my_cand;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      incl += lane >= o ? y : 0u;
+    }
+    const uint32_t wtot = __shfl_sync(0xffffffffu, incl, 31);
     uint32_t base = 0u;
-    if (lane == leader) base = atomicAdd(&sm.cand_n, static_cast<uint32_t>(__popc(m)));
-    base = __shfl_sync(0xffffffffu, base, leader);
-    if (is_cand) {
-      const uint32_t slot = base + __popc(m & ((1u << lane) - 1u));
-      if (slot < static_cast<uint32_t>(kClusterCandCap))
+    if (lane == 31 && wtot) base = atomicAdd(&sm.cand_n, wtot);
+    uint32_t slot = __shfl_sync(0xffffffffu, base, 31) + incl - my_cand;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      const int li = e * NT + tid;
+      const bool is_cand = c0 + li < V && QSA_BIN(e) == thr_bin;
+      if (is_cand && slot < static_cast<uint32_t>(kClusterCandCap))
         sm.cand[slot] = make_uint2(QSA_KEY(e), static_cast<uint32_t>(li));
+      slot += is_cand ? 1u : 0u;
     }
   }
   my_sure = __reduce_add_sync(0xffffffffu, my_sure);
@@ -455,21 +464,32 @@ __global__ void __launch_bounds__(kClusterThreads) cluster_select_kernel(const f
   const uint32_t thr_key = prefix;
   const uint32_t take_eq = need;  // lowest-index cells with key == thr_key to keep
 
-  // ---- mark this CTA's cells
-  for (int i = tid; i < WORDS; i += NT) {
-    sm.selb[i] = 0u;
-    sm.eqb[i] = 0u;
-  }
-  __syncthreads();
+  // ---- mark this CTA's cells.  A higher key is a larger score and equal keys share a
+  // bin, so the cells kept are those with key > thr_key and the ties key == thr_key.
+  // Word e * (NT / 32) + w of a bitmap holds element e of warp w's 32 threads: one
+  // ballot each, kept by lane e % 32 and stored once (no clearing, no atomics).
+  {
+    constexpr int H = (PER + 31) / 32;
+    uint32_t w_sel[H], w_eq[H];
 #pragma unroll
-  for (int e = 0; e < PER; ++e) {
-    const int li = e * NT + tid;
-    if (c0 + li >= V) continue;
-    const uint32_t b = QSA_BIN(e);
-    if (b < thr_bin) continue;
-    const uint32_t k = QSA_KEY(e);
-    if (b > thr_bin || k > thr_key) atomicOr(&sm.selb[li >> 5], 1u << (li & 31));
-    else if (k == thr_key) atomicOr(&sm.eqb[li >> 5], 1u << (li & 31));
+    for (int h = 0; h < H; ++h) w_sel[h] = w_eq[h] = 0u;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      const bool valid = c0 + e * NT + tid < V;
+      const uint32_t k = QSA_KEY(e);
+      const uint32_t bs = __ballot_sync(0xffffffffu, valid && k > thr_key);
+      const uint32_t be = __ballot_sync(0xffffffffu, valid && k == thr_key);
+      w_sel[e >> 5] = lane == (e & 31) ? bs : w_sel[e >> 5];
+      w_eq[e >> 5] = lane == (e & 31) ? be : w_eq[e >> 5];
+    }
+#pragma unroll
+    for (int h = 0; h < H; ++h) {
+      const int e = h * 32 + lane;
+      if (e < PER) {
+        sm.selb[e * (NT / 32) + (tid >> 5)] = w_sel[h];
+        sm.eqb[e * (NT / 32) + (tid >> 5)] = w_eq[h];
+      }
+    }
   }
   __syncthreads();
   const int per = (WORDS + NT - 1) / NT;
