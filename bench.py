@@ -504,8 +504,9 @@ def kernel_times(qsa, torch, spec, caches, wl, q, iq, iw, ws, dev, stream, reps)
 
 
 def auto_nsplit(rows, top_k):
-    """The library's automatic split count (qsa_api.cu): about 256 CTAs in all."""
-    want = 128 // rows
+    """The library's automatic split count (qsa_api.cu): 32 pieces for up to 8 rows,
+    about 256 CTAs in all beyond."""
+    want = 32 if rows <= 8 else 128 // rows
     return max(1, min(64, max(1, top_k // 32), want))
 
 

@@ -182,11 +182,12 @@ struct StepPlan {
 };
 
 int auto_nsplit(int rows, int top_k) {
-  // About 256 (row, KV head, split) CTAs, pieces of at least 32 cells: on a B200
-  // the attention plus the merge of a decode step of 1-8 rows is fastest there
-  // (more splits shorten the gathers but lengthen the merge); large prefill
-  // chunks need no splits.
-  const int want = 128 / rows;
+  // Pieces of at least 32 cells.  Up to 8 rows: 32 pieces.  On a B200 the
+  // graph-replayed decode step of 1-8 rows at 64K cells and top_k = 2048 was
+  // fastest there or within noise of it for every row count (more pieces
+  // shorten the gathers but lengthen the merge).  More rows: about 256 (row,
+  // KV head, split) CTAs; large prefill chunks need no splits.
+  const int want = rows <= QSA_MAX_DECODE ? 32 : 128 / rows;
   return std::max(1, std::min({QSA_MAX_SPLITS, std::max(1, top_k / 32), want}));
 }
 
