@@ -122,7 +122,10 @@ int qsa_cache_write(const qsa_cache* cache, int pos0, int n, const float* k, con
  * over the selected cells, computed as nsplit pieces of the selected list
  * (ceil(top_k / nsplit) entries each) merged by log-sum-exp (qsa_merge,
  * same page, section 2).  nsplit = 0 lets the library choose; the result
- * does not depend on nsplit beyond rounding.
+ * does not depend on nsplit beyond rounding.  When every token sees at most
+ * top_k cells (L <= top_k), all visible cells are selected: the call skips
+ * the scores and the selection (the dense path for short contexts, the pages'
+ * qsa_flash case) and returns the same result and ids.
  *   out      fp32 [n][24][256]
  *   ids_out  int32 [n][top_k] or NULL: the selected cells, ascending, -1 padded
  *   ws       device workspace of at least qsa_workspace_bytes(...) bytes
@@ -139,7 +142,8 @@ int qsa_decode(const qsa_cache* cache, int L, int n, const float* q, const uint1
  * what changed, items 1-2; "Round 5 Track C Report ...", section 2.1).  Row t
  * sees cells [0, pos0 + t]; the chunk's own cells must already be written.
  * Arguments as qsa_decode with n -> T (q [T][24][256], iq [T][4][64],
- * iw [T][4], out [T][24][256], ids_out [T][top_k] or NULL).
+ * iw [T][4], out [T][24][256], ids_out [T][top_k] or NULL).  A chunk with
+ * pos0 + T <= top_k takes the dense path, as qsa_decode does.
  * Requires 0 <= pos0, 1 <= T, pos0 + T <= max_cells.
  */
 int qsa_prefill_chunk(const qsa_cache* cache, int pos0, int T, const float* q,

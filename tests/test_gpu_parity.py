@@ -443,6 +443,57 @@ def test_decode_dense_when_few_cells(gpu):
         assert rel_err(out[i], oracle.dense_attn_row(wl.cache, V, wl.q[i], wl.scale)) <= OUT_TOL
 
 
+@pytest.mark.parametrize("n,nsplit", [(1, 1), (3, 5), (8, 32), (8, 0)])
+def test_decode_short_context_bit_equal(gpu, n, nsplit):
+    # every row sees at most top_k cells: the step skips the scores and the selection and
+    # walks cells 0 .. V - 1 itself, bit-equal to the selection's list run by qsa_attn
+    qsa = gpu
+    top_k = 512
+    wl = synth.make_workload(1, n=n, cells=top_k)
+    cache, q, iq, iw = dev_inputs(qsa, wl)
+    ids = torch.full((n, top_k), 7, dtype=torch.int32, device=DEV)
+    out = qsa.decode(cache, wl.L, q, iq, iw, top_k, nsplit, wl.scale, ids_out=ids).cpu().numpy()
+    ns = nsplit or qsa_auto_nsplit(n, top_k)
+    ref_ids = -np.ones((n, top_k), np.int32)
+    for i in range(n):
+        ref_ids[i, :wl.L - n + 1 + i] = np.arange(wl.L - n + 1 + i)
+    assert np.array_equal(ids.cpu().numpy(), ref_ids)
+    res = qsa.attn(cache, q, torch.from_numpy(ref_ids).to(DEV), ns, wl.scale)
+    two = (res if ns == 1 else qsa.merge(res)).cpu().numpy()
+    assert np.array_equal(out.view(np.uint32), two.view(np.uint32))
+    for i in range(n):
+        assert rel_err(out[i], oracle.dense_attn_row(wl.cache, wl.L - n + 1 + i, wl.q[i], wl.scale)) <= OUT_TOL
+
+
+@pytest.mark.parametrize("extra", [0, 1])
+def test_decode_short_context_boundary(gpu, extra):
+    # the last row sees top_k cells (implicit list) or top_k + 1 (scores and selection)
+    wl = synth.make_workload(1, n=4, cells=300 + extra)
+    wl.top_k = 300
+    _decode_case(gpu, wl, 3)
+
+
+@pytest.mark.parametrize("T", [4, 16])
+def test_prefill_short_context(gpu, T):
+    # a chunk inside the first top_k cells: every row attends to all the cells it sees
+    qsa = gpu
+    top_k, pos0 = 512, 100
+    wl = synth.make_workload(3, cells=pos0 + T, rows=T)
+    cache, q, iq, iw = dev_inputs(qsa, wl)
+    ids = torch.empty(T, top_k, dtype=torch.int32, device=DEV)
+    out = qsa.prefill_chunk(cache, pos0, q, iq, iw, top_k, wl.scale, ids_out=ids).cpu().numpy()
+    ids = ids.cpu().numpy()
+    for t in range(T):
+        V = pos0 + t + 1
+        assert np.array_equal(ids[t, :V], np.arange(V)) and np.all(ids[t, V:] == -1)
+        assert rel_err(out[t], oracle.dense_attn_row(wl.cache, V, wl.q[t], wl.scale)) <= OUT_TOL
+
+
+def qsa_auto_nsplit(rows, top_k):
+    import bench
+    return bench.auto_nsplit(rows, top_k)
+
+
 def test_decode_nsplit_invariance(gpu):
     qsa = gpu
     wl = synth.make_workload(1, n=2, cells=6000)

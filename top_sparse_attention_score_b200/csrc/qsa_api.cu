@@ -104,12 +104,12 @@ int prepare_device() {
   cudaError_t e = cudaFuncSetAttribute(qsa::topk_final_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        2 * (qsa::kMaxWindowBits / 32) * 4);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(qsa::attn_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(sizeof(qsa::AttnSmem<4>)));
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(qsa::attn_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(sizeof(qsa::AttnSmem<2>)));
+#define QSA_ATTN_SMEM(W, ALL)                                                                   \
+  if (e == cudaSuccess)                                                                         \
+    e = cudaFuncSetAttribute(qsa::attn_kernel<W, ALL>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             static_cast<int>(sizeof(qsa::AttnSmem<W>)));
+  QSA_ATTN_SMEM(4, false) QSA_ATTN_SMEM(4, true) QSA_ATTN_SMEM(2, false) QSA_ATTN_SMEM(2, true)
+#undef QSA_ATTN_SMEM
 #define QSA_CLUSTER_SMEM(P)                                                                     \
   if (e == cudaSuccess)                                                                         \
     e = cudaFuncSetAttribute(qsa::cluster_select_kernel<P>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
@@ -374,8 +374,11 @@ int launch_selection(const float* scores, int64_t ld, int rows, int vis0, int to
   return launch_topk(scores, ld, rows, vis0, top_k, ws, p, ids, s);
 }
 
+// ids == NULL: every row's list is all its visible cells (row r sees dense_vis0 + r <= top_k),
+// copied to ids_fill when that is not NULL.
 int launch_attn(const qsa_cache* c, int rows, const float* q, const int32_t* ids, int top_k,
-                int nsplit, float scale, float* part, float* out, cudaStream_t s) {
+                int nsplit, float scale, float* part, float* out, cudaStream_t s, int dense_vis0 = 0,
+                int32_t* ids_fill = nullptr) {
   qsa::AttnArgs a;
   a.k = c->k;
   a.v = c->v;
@@ -390,10 +393,16 @@ int launch_attn(const qsa_cache* c, int rows, const float* q, const int32_t* ids
   a.scale_log2 = scale * 1.4426950408889634f;
   a.part = part;
   a.out = out;
-  if (rows <= QSA_MAX_DECODE)
-    launch_pdl(qsa::attn_kernel<4>, dim3(nsplit, QSA_HKV, rows), dim3(128), sizeof(qsa::AttnSmem<4>), s, a);
-  else
-    launch_pdl(qsa::attn_kernel<2>, dim3(nsplit, QSA_HKV, rows), dim3(64), sizeof(qsa::AttnSmem<2>), s, a);
+  a.dense_vis0 = dense_vis0;
+  a.ids_fill = ids_fill;
+  const dim3 grid(nsplit, QSA_HKV, rows);
+  if (rows <= QSA_MAX_DECODE) {
+    if (ids) launch_pdl(qsa::attn_kernel<4, false>, grid, dim3(128), sizeof(qsa::AttnSmem<4>), s, a);
+    else launch_pdl(qsa::attn_kernel<4, true>, grid, dim3(128), sizeof(qsa::AttnSmem<4>), s, a);
+  } else {
+    if (ids) launch_pdl(qsa::attn_kernel<2, false>, grid, dim3(64), sizeof(qsa::AttnSmem<2>), s, a);
+    else launch_pdl(qsa::attn_kernel<2, true>, grid, dim3(64), sizeof(qsa::AttnSmem<2>), s, a);
+  }
   return launched("attn_kernel");
 }
 
@@ -421,9 +430,15 @@ int run_step(const qsa_cache* c, int rows, int vis0, int ncells, const float* q,
   float* scores = reinterpret_cast<float*>(base + p.scores);
   int32_t* ids = ids_out ? ids_out : reinterpret_cast<int32_t*>(base + p.ids);
   float* part = reinterpret_cast<float*>(base + p.part);
-  if ((r = launch_index_score(c, rows, ncells, iq, iw, scores, p.ld, s))) return r;
-  if ((r = launch_selection(scores, p.ld, rows, vis0, top_k, base, p.topk, ids, s))) return r;
-  if ((r = launch_attn(c, rows, q, ids, top_k, nsplit, scale, part, out, s))) return r;
+  if (vmax <= top_k) {
+    // Every row sees at most top_k cells, so the selection would keep all of them in
+    // order: no scores, no selection; the attention walks cells 0 .. V - 1 itself.
+    if ((r = launch_attn(c, rows, q, nullptr, top_k, nsplit, scale, part, out, s, vis0, ids_out))) return r;
+  } else {
+    if ((r = launch_index_score(c, rows, ncells, iq, iw, scores, p.ld, s))) return r;
+    if ((r = launch_selection(scores, p.ld, rows, vis0, top_k, base, p.topk, ids, s))) return r;
+    if ((r = launch_attn(c, rows, q, ids, top_k, nsplit, scale, part, out, s))) return r;
+  }
   if (nsplit > 1 && (r = launch_merge(part, rows, nsplit, out, s))) return r;
   return ok();
 }

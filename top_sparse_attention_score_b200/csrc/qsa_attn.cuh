@@ -56,7 +56,7 @@ struct AttnArgs {
   const __half* ks;
   const __half* vs;
   const float* q;     // [rows][24][256]
-  const int* ids;     // [rows][top_k]
+  const int* ids;     // [rows][top_k]; NULL: row r's list is cells 0 .. dense_vis0 + r - 1, -1 padded
   int top_k;
   int max_cells;      // ids outside [0, max_cells) are treated as empty slots
   int nsplit;
@@ -64,10 +64,20 @@ struct AttnArgs {
   float scale_log2;   // softmax scale * log2(e)
   float* part;        // [rows][24][nsplit][258] when nsplit > 1
   float* out;         // [rows][24][256] when nsplit == 1
+  int dense_vis0;     // ids == NULL: cells row 0 sees (row r sees dense_vis0 + r <= top_k)
+  int* ids_fill;      // ids == NULL: optional [rows][top_k] copy of the implicit lists
 };
 
-template <int NT>
-__device__ __forceinline__ void attn_issue(AttnStage& st, const AttnArgs& a, const int* rid, int pos0,
+// Cell of list position p < end: ids[p], or with the implicit list (kAll) p itself below dv.
+template <bool kAll>
+__device__ __forceinline__ int attn_cell(const int* rid, int dv, int p, int end) {
+  if (p >= end) return -1;
+  if constexpr (kAll) return p < dv ? p : -1;
+  else return __ldg(rid + p);
+}
+
+template <int NT, bool kAll>
+__device__ __forceinline__ void attn_issue(AttnStage& st, const AttnArgs& a, const int* rid, int dv, int pos0,
                                            int end, int kvh) {
   const int tid = threadIdx.x;
   // K and V rows: 32 cells x 16 chunks of 16 bytes each, 512 / NT + 512 / NT per thread.
@@ -76,7 +86,7 @@ __device__ __forceinline__ void attn_issue(AttnStage& st, const AttnArgs& a, con
     const int chunk = tid + NT * u;
     const int i = chunk >> 4, part = chunk & 15;
     const int p = pos0 + i;
-    int cell = p < end ? __ldg(rid + p) : -1;
+    int cell = attn_cell<kAll>(rid, dv, p, end);
     const bool ok = cell >= 0 && cell < a.max_cells;
     if (!ok) cell = 0;
     const size_t row = (static_cast<size_t>(cell) * kHKV + kvh) * kD + part * 16;
@@ -86,7 +96,7 @@ __device__ __forceinline__ void attn_issue(AttnStage& st, const AttnArgs& a, con
   if (tid < 2 * kAttnCells) {  // scales: 64 rows of 16 bytes
     const int i = tid & 31;
     const int p = pos0 + i;
-    int cell = p < end ? __ldg(rid + p) : -1;
+    int cell = attn_cell<kAll>(rid, dv, p, end);
     const bool ok = cell >= 0 && cell < a.max_cells;
     if (tid < kAttnCells) st.valid[i] = ok;
     if (!ok) cell = 0;
@@ -97,7 +107,8 @@ __device__ __forceinline__ void attn_issue(AttnStage& st, const AttnArgs& a, con
 }
 
 // grid: (nsplit, 2, rows); block: 32 * W threads; dynamic smem: sizeof(AttnSmem<W>).
-template <int W>
+// kAll: a.ids is NULL and every row's list is all its visible cells.
+template <int W, bool kAll>
 __global__ void __launch_bounds__(32 * W) attn_kernel(AttnArgs a) {
   constexpr int NT = 32 * W;
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -107,7 +118,8 @@ __global__ void __launch_bounds__(32 * W) attn_kernel(AttnArgs a) {
   const int g = lane >> 2, t = lane & 3;
   const int beg = min(a.top_k, split * a.piece);
   const int end = min(a.top_k, beg + a.piece);
-  const int* rid = a.ids + static_cast<size_t>(row) * a.top_k;
+  const int* rid = kAll ? nullptr : a.ids + static_cast<size_t>(row) * a.top_k;
+  const int dv = kAll ? a.dense_vis0 + row : 0;  // implicit list: every visible cell
   const int nblk = (end - beg + kAttnCells - 1) / kAttnCells;
   griddep_launch();
 
@@ -142,9 +154,14 @@ __global__ void __launch_bounds__(32 * W) attn_kernel(AttnArgs a) {
 
   // The ids come from the selection kernel: wait for it before the first gather.
   griddep_wait();
+  if constexpr (kAll) {
+    if (a.ids_fill && kvh == 0)  // this piece of the implicit list, for the caller
+      for (int p = beg + static_cast<int>(threadIdx.x); p < end; p += NT)
+        a.ids_fill[static_cast<size_t>(row) * a.top_k + p] = p < dv ? p : -1;
+  }
 #pragma unroll
   for (int st = 0; st < kAttnStages - 1; ++st) {
-    if (st < nblk) attn_issue<NT>(sm.st[st], a, rid, beg + st * kAttnCells, end, kvh);
+    if (st < nblk) attn_issue<NT, kAll>(sm.st[st], a, rid, dv, beg + st * kAttnCells, end, kvh);
     cp_async_commit();
   }
 
@@ -164,7 +181,7 @@ __global__ void __launch_bounds__(32 * W) attn_kernel(AttnArgs a) {
   for (int b = 0; b < nblk; ++b) {
     // refill the stage block b - 1 used (every warp finished it at the last barrier)
     const int nb = b + kAttnStages - 1;
-    if (nb < nblk) attn_issue<NT>(sm.st[nb % kAttnStages], a, rid, beg + nb * kAttnCells, end, kvh);
+    if (nb < nblk) attn_issue<NT, kAll>(sm.st[nb % kAttnStages], a, rid, dv, beg + nb * kAttnCells, end, kvh);
     cp_async_commit();
     cp_async_wait<kAttnStages - 1>();
     __syncthreads();
