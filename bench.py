@@ -386,16 +386,19 @@ def run_cuda(args, spec: Spec):
     for n in spec.ns:
         d2h += n * 24 * 256 * 4
 
+    # each call's row views, made once (a caller with fixed buffers holds them)
+    views = {n: (kd[:n], vd[:n], keyd[:n], qd[:n], iqd[:n], iwd[:n], out[:n], out_h[:n]) for n in spec.ns}
+
     def e2e_step(i):
         for dst, src in ((qd, q_h), (iqd, iq_h), (iwd, iw_h), (kd, kk_h), (vd, vv_h), (keyd, key_hh)):
             dst.copy_(src, non_blocking=True)
         c = caches[i % ROTATE]
         for n in spec.ns:
             if spec.kind == "decode":
-                qsa.cache_write(c, spec.L - n, kd[:n], vd[:n], keyd[:n])
-                qsa.decode(c, spec.L, qd[:n], iqd[:n], iwd[:n], spec.top_k, spec.nsplit, wl.scale,
-                           ws=ws, out=out[:n])
-                out_h[:n].copy_(out[:n], non_blocking=True)
+                kn_, vn_, keyn_, qn_, iqn_, iwn_, outn_, outhn_ = views[n]
+                qsa.cache_write(c, spec.L - n, kn_, vn_, keyn_)
+                qsa.decode(c, spec.L, qn_, iqn_, iwn_, spec.top_k, spec.nsplit, wl.scale, ws=ws, out=outn_)
+                outhn_.copy_(outn_, non_blocking=True)
             else:
                 qsa.cache_write(c, spec.pos0, kd, vd, keyd)
                 qsa.prefill_chunk(c, spec.pos0, qd, iqd, iwd, spec.top_k, wl.scale, ws=ws, out=out)

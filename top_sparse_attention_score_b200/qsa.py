@@ -82,12 +82,21 @@ def _check(code: int) -> None:
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    # the signatures declare c_void_p: a plain int (or None for NULL) needs no wrapper
+    return None if t is None else t.data_ptr()
+
+
+# The raw handle of torch's current stream on the current device, without building
+# a torch.cuda.Stream object per call (the public path below is the fallback).
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
 
 
 def _stream(stream):
-    s = torch.cuda.current_stream() if stream is None else stream
-    return ctypes.c_void_p(s.cuda_stream)
+    if stream is not None:
+        return stream.cuda_stream
+    if _raw_stream is not None:
+        return _raw_stream(torch.cuda.current_device())
+    return torch.cuda.current_stream().cuda_stream
 
 
 def _dev(t: torch.Tensor, dtype, name: str):
@@ -137,6 +146,18 @@ class DeviceCache:
         return CacheStruct(self.k.data_ptr(), self.v.data_ptr(), self.ks.data_ptr(),
                            self.vs.data_ptr(), self.idx_key.data_ptr(), self.cells)
 
+    def ref(self) -> int:
+        """Address of a qsa_cache for this cache, rebuilt (and checked again) whenever
+        an array's storage or the cell count differs from the last call."""
+        key = (self.k.data_ptr(), self.v.data_ptr(), self.ks.data_ptr(), self.vs.data_ptr(),
+               self.idx_key.data_ptr(), self.k.shape[0])
+        held = self.__dict__.get("_held")
+        if held is None or held[0] != key:
+            cs = self.struct()
+            held = (key, cs, ctypes.addressof(cs))
+            self.__dict__["_held"] = held
+        return held[2]
+
 
 def workspace_bytes(mode: int, rows: int, L: int, top_k: int, nsplit: int = 0) -> int:
     return int(load().qsa_workspace_bytes(mode, rows, L, top_k, nsplit))
@@ -151,8 +172,7 @@ def workspace(nbytes: int, device="cuda") -> torch.Tensor:
 
 
 def cache_write(cache: DeviceCache, pos0: int, k, v, key, stream=None) -> None:
-    cs = cache.struct()
-    _check(load().qsa_cache_write(ctypes.byref(cs), pos0, k.shape[0],
+    _check(load().qsa_cache_write(cache.ref(), pos0, k.shape[0],
                                   _ptr(_dev(k, torch.float32, "k")), _ptr(_dev(v, torch.float32, "v")),
                                   _ptr(_dev(key, torch.float16, "key")), _stream(stream)))
 
@@ -164,8 +184,7 @@ def decode(cache: DeviceCache, L: int, q, iq, iw, top_k: int, nsplit: int = 0, s
         ws = workspace(workspace_bytes(MODE_DECODE, n, L, top_k, nsplit), q.device)
     if out is None:
         out = torch.empty(n, HQ, D, dtype=torch.float32, device=q.device)
-    cs = cache.struct()
-    _check(load().qsa_decode(ctypes.byref(cs), L, n, _ptr(_dev(q, torch.float32, "q")),
+    _check(load().qsa_decode(cache.ref(), L, n, _ptr(_dev(q, torch.float32, "q")),
                              _ptr(_dev(iq, torch.float16, "iq")), _ptr(_dev(iw, torch.float32, "iw")),
                              top_k, nsplit, scale, _ptr(ws), ws.numel(), _ptr(out),
                              _ptr(None if ids_out is None else _dev(ids_out, torch.int32, "ids_out")),
@@ -180,8 +199,7 @@ def prefill_chunk(cache: DeviceCache, pos0: int, q, iq, iw, top_k: int, scale: f
         ws = workspace(workspace_bytes(MODE_PREFILL, T, pos0 + T, top_k), q.device)
     if out is None:
         out = torch.empty(T, HQ, D, dtype=torch.float32, device=q.device)
-    cs = cache.struct()
-    _check(load().qsa_prefill_chunk(ctypes.byref(cs), pos0, T, _ptr(_dev(q, torch.float32, "q")),
+    _check(load().qsa_prefill_chunk(cache.ref(), pos0, T, _ptr(_dev(q, torch.float32, "q")),
                                     _ptr(_dev(iq, torch.float16, "iq")),
                                     _ptr(_dev(iw, torch.float32, "iw")), top_k, scale, _ptr(ws),
                                     ws.numel(), _ptr(out),
@@ -195,8 +213,7 @@ def index_score(cache: DeviceCache, iq, iw, ncells: int, scores=None, stream=Non
     if scores is None:
         ld = (ncells + 3) // 4 * 4
         scores = torch.empty(rows, ld, dtype=torch.float32, device=iq.device)
-    cs = cache.struct()
-    _check(load().qsa_index_score(ctypes.byref(cs), rows, ncells, _ptr(_dev(iq, torch.float16, "iq")),
+    _check(load().qsa_index_score(cache.ref(), rows, ncells, _ptr(_dev(iq, torch.float16, "iq")),
                                   _ptr(_dev(iw, torch.float32, "iw")),
                                   _ptr(_dev(scores, torch.float32, "scores")), scores.shape[1],
                                   _stream(stream)))
@@ -221,8 +238,7 @@ def attn(cache: DeviceCache, q, ids, nsplit: int = 1, scale: float = 1 / 16, par
         out = torch.empty(rows, HQ, D, dtype=torch.float32, device=q.device)
     if nsplit > 1 and part is None:
         part = torch.empty(rows, HQ, nsplit, PART_STRIDE, dtype=torch.float32, device=q.device)
-    cs = cache.struct()
-    _check(load().qsa_attn(ctypes.byref(cs), rows, _ptr(_dev(q, torch.float32, "q")),
+    _check(load().qsa_attn(cache.ref(), rows, _ptr(_dev(q, torch.float32, "q")),
                            _ptr(_dev(ids, torch.int32, "ids")), top_k, nsplit, scale, _ptr(part),
                            _ptr(out), _stream(stream)))
     return out if nsplit == 1 else part
