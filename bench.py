@@ -21,6 +21,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -162,8 +163,13 @@ def peaks():
 
 
 def source_hash(kernel: str) -> str:
+    """Hash of the kernel's source without comments and blank space: edits to comments
+    alone keep the recorded traffic, any change to the code drops it."""
     src = os.path.join(ROOT, "top_sparse_attention_score_b200", "csrc", KERNEL_SOURCES[kernel])
-    return hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    code = re.sub(r"/\*.*?\*/", "", open(src).read(), flags=re.S)
+    code = re.sub(r"//[^\n]*", "", code)
+    code = "\n".join(line.strip() for line in code.splitlines() if line.strip())
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
 def traffic_for(kernel: str, workload: str):

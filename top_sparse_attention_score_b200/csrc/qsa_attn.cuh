@@ -19,7 +19,10 @@
 //    MMA; the per-32 V scale multiplies the fp16 V operand.  Q and P are fp16;
 //  * the reference maximum of the online softmax moves only when a block
 //    exceeds it by more than 2^8, so P stays <= 256 and most blocks skip the
-//    rescale of O; split partials are reported against the true maximum.
+//    rescale of O; split partials are reported against the true maximum;
+//  * a second instantiation (kAll) serves rows that see at most top_k cells:
+//    the selection would keep all of them, so list position p is cell p and
+//    no ids are read (the whole-step calls then launch no score or selection).
 #pragma once
 
 #include "qsa_common.cuh"
