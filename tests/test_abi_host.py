@@ -117,3 +117,20 @@ def test_bench_split_rule_matches_the_library(lib):
             other = bench.auto_nsplit(n, k) + 1
             if other <= 64:
                 assert auto != lib.qsa_workspace_bytes(0, n, 65536, k, other), (n, k)
+
+
+def test_traffic_hash_follows_code_not_comments(tmp_path, monkeypatch):
+    """A recorded DRAM-traffic figure stays valid through comment edits of its kernel's
+    source and is dropped by any change to the code."""
+    import bench
+    csrc = tmp_path / "top_sparse_attention_score_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    src = csrc / bench.KERNEL_SOURCES["merge_kernel"]
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    base = "// header\n#pragma once\n/* block\n comment */\nint f(int x) {  // trailing\n  return x + 1;\n}\n"
+    src.write_text(base)
+    h0 = bench.source_hash("merge_kernel")
+    src.write_text(base.replace("// trailing", "// reworded").replace("block\n comment", "other text") + "\n\n")
+    assert bench.source_hash("merge_kernel") == h0
+    src.write_text(base.replace("x + 1", "x + 2"))
+    assert bench.source_hash("merge_kernel") != h0
