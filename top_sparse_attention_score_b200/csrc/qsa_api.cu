@@ -47,11 +47,16 @@ int ok() {
   return QSA_OK;
 }
 
-// Count a launch and turn a launch error into QSA_ERR_CUDA.
-int launched(const char* what) {
+// Count a launch and turn the error its launch call returned into QSA_ERR_CUDA.
+// Only a failed launch clears the runtime's last-error state (which it set): an
+// error left there by the caller's own earlier work is neither taken for this
+// launch's nor cleared.
+int launched(const char* what, cudaError_t e) {
   g_launches.fetch_add(1, std::memory_order_relaxed);
-  const cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(QSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  }
   return QSA_OK;
 }
 
@@ -273,8 +278,8 @@ int launch_score_gemm(const qsa_cache* c, int rows, int ncells, const uint16_t* 
   const int items = ((rows + qsa::kGemmTokens - 1) / qsa::kGemmTokens) *
                     ((ncells + qsa::kGemmCells - 1) / qsa::kGemmCells);
   const dim3 grid(std::max(1, std::min(items, sm_count())));
-  launch_pdl(qsa::score_gemm_kernel, grid, dim3(qsa::kGemmThreads), qsa::kGemmSmemRequest, s, tkey, tiq, tout, a);
-  return launched("score_gemm_kernel");
+  return launched("score_gemm_kernel", launch_pdl(qsa::score_gemm_kernel, grid, dim3(qsa::kGemmThreads),
+                                                  qsa::kGemmSmemRequest, s, tkey, tiq, tout, a));
 }
 
 int launch_index_score(const qsa_cache* c, int rows, int ncells, const uint16_t* iq,
@@ -282,33 +287,32 @@ int launch_index_score(const qsa_cache* c, int rows, int ncells, const uint16_t*
   if (rows > qsa::kScoreRowsPerCta) return launch_score_gemm(c, rows, ncells, iq, iw, scores, ld, s);
   const dim3 grid((ncells + qsa::kScoreCellsPerCta - 1) / qsa::kScoreCellsPerCta,
                   (rows + qsa::kScoreRowsPerCta - 1) / qsa::kScoreRowsPerCta);
-  launch_pdl(qsa::index_score_kernel, grid, dim3(128), 0, s,
-             reinterpret_cast<const __half*>(c->idx_key), ncells, reinterpret_cast<const __half*>(iq),
-             iw, rows, scores, ld);
-  return launched("index_score_kernel");
+  return launched("index_score_kernel",
+                  launch_pdl(qsa::index_score_kernel, grid, dim3(128), 0, s,
+                             reinterpret_cast<const __half*>(c->idx_key), ncells,
+                             reinterpret_cast<const __half*>(iq), iw, rows, scores, ld));
 }
 
 int launch_zero(void* ws, const TopkPlan& p, cudaStream_t s) {
   // hist and ctr are adjacent up to alignment padding; zero both regions.
   const int64_t nzero = static_cast<int64_t>((p.sure - p.hist) / 4);
   const int zblocks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(592, (nzero + 255) / 256)));
-  launch_pdl(qsa::topk_zero_kernel, dim3(zblocks), dim3(256), 0, s,
-             reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + p.hist), nzero);
-  return launched("topk_zero_kernel");
+  return launched("topk_zero_kernel",
+                  launch_pdl(qsa::topk_zero_kernel, dim3(zblocks), dim3(256), 0, s,
+                             reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + p.hist), nzero));
 }
 
 int launch_filter_final(const float* scores, int64_t ld, int rows, int vis0, int top_k,
                         const qsa::TopkWs& w, int32_t* ids, cudaStream_t s) {
   const int vmax = vis0 + rows - 1;
   const dim3 grid((vmax + qsa::kTopkChunk - 1) / qsa::kTopkChunk, rows);
-  launch_pdl(qsa::topk_filter_kernel, grid, dim3(qsa::kTopkThreads), 0, s, scores, ld, vis0, top_k, w);
-  int r = launched("topk_filter_kernel");
+  int r = launched("topk_filter_kernel", launch_pdl(qsa::topk_filter_kernel, grid, dim3(qsa::kTopkThreads), 0,
+                                                    s, scores, ld, vis0, top_k, w));
   if (r) return r;
   const int win = std::min(qsa::kMaxWindowBits, static_cast<int>(align_up(vmax, 32)));
   const size_t smem = 2 * static_cast<size_t>(win / 32) * 4;
-  launch_pdl(qsa::topk_final_kernel, dim3(rows), dim3(qsa::kFinalThreads), smem, s, scores, ld, vis0, top_k,
-             w, win, ids);
-  return launched("topk_final_kernel");
+  return launched("topk_final_kernel", launch_pdl(qsa::topk_final_kernel, dim3(rows), dim3(qsa::kFinalThreads),
+                                                  smem, s, scores, ld, vis0, top_k, w, win, ids));
 }
 
 // Selection over given scores: zero, histogram (+ thresholds), filter, final.
@@ -319,8 +323,9 @@ int launch_topk(const float* scores, int64_t ld, int rows, int vis0, int top_k, 
   int r = launch_zero(ws, p, s);
   if (r) return r;
   const dim3 grid((vmax + qsa::kTopkChunk - 1) / qsa::kTopkChunk, rows);
-  launch_pdl(qsa::topk_hist_kernel, grid, dim3(qsa::kTopkThreads), 0, s, scores, ld, vis0, top_k, w);
-  if ((r = launched("topk_hist_kernel"))) return r;
+  if ((r = launched("topk_hist_kernel", launch_pdl(qsa::topk_hist_kernel, grid, dim3(qsa::kTopkThreads), 0, s,
+                                                   scores, ld, vis0, top_k, w))))
+    return r;
   return launch_filter_final(scores, ld, rows, vis0, top_k, w, ids, s);
 }
 
@@ -342,8 +347,8 @@ int launch_cluster_select_per(const float* scores, int64_t ld, int rows, int vis
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  cudaLaunchKernelEx(&cfg, qsa::cluster_select_kernel<PER>, scores, ld, vis0, top_k, ids);
-  return launched("cluster_select_kernel");
+  return launched("cluster_select_kernel",
+                  cudaLaunchKernelEx(&cfg, qsa::cluster_select_kernel<PER>, scores, ld, vis0, top_k, ids));
 }
 
 // Longest row the decode selection gives to one cluster (16 cells per thread); longer
@@ -396,19 +401,20 @@ int launch_attn(const qsa_cache* c, int rows, const float* q, const int32_t* ids
   a.dense_vis0 = dense_vis0;
   a.ids_fill = ids_fill;
   const dim3 grid(nsplit, QSA_HKV, rows);
+  cudaError_t e;
   if (rows <= QSA_MAX_DECODE) {
-    if (ids) launch_pdl(qsa::attn_kernel<4, false>, grid, dim3(128), sizeof(qsa::AttnSmem<4>), s, a);
-    else launch_pdl(qsa::attn_kernel<4, true>, grid, dim3(128), sizeof(qsa::AttnSmem<4>), s, a);
+    if (ids) e = launch_pdl(qsa::attn_kernel<4, false>, grid, dim3(128), sizeof(qsa::AttnSmem<4>), s, a);
+    else e = launch_pdl(qsa::attn_kernel<4, true>, grid, dim3(128), sizeof(qsa::AttnSmem<4>), s, a);
   } else {
-    if (ids) launch_pdl(qsa::attn_kernel<2, false>, grid, dim3(64), sizeof(qsa::AttnSmem<2>), s, a);
-    else launch_pdl(qsa::attn_kernel<2, true>, grid, dim3(64), sizeof(qsa::AttnSmem<2>), s, a);
+    if (ids) e = launch_pdl(qsa::attn_kernel<2, false>, grid, dim3(64), sizeof(qsa::AttnSmem<2>), s, a);
+    else e = launch_pdl(qsa::attn_kernel<2, true>, grid, dim3(64), sizeof(qsa::AttnSmem<2>), s, a);
   }
-  return launched("attn_kernel");
+  return launched("attn_kernel", e);
 }
 
 int launch_merge(const float* part, int rows, int nsplit, float* out, cudaStream_t s) {
-  launch_pdl(qsa::merge_kernel, dim3(rows * QSA_HQ), dim3(256), 0, s, part, nsplit, out);
-  return launched("merge_kernel");
+  return launched("merge_kernel", launch_pdl(qsa::merge_kernel, dim3(rows * QSA_HQ), dim3(256), 0, s, part,
+                                             nsplit, out));
 }
 
 // The whole step for `rows` query rows; row r sees vis0 + r cells of ncells.
@@ -471,11 +477,13 @@ int qsa_cache_write(const qsa_cache* cache, int pos0, int n, const float* k, con
   if (n < 1 || pos0 < 0 || static_cast<int64_t>(pos0) + n > cache->max_cells)
     return fail(QSA_ERR_ARG, "cells [%d, %d + %d) outside the cache of %d", pos0, pos0, n,
                 cache->max_cells);
-  launch_pdl(qsa::cache_write_kernel, dim3(n, QSA_HKV, 2), dim3(256), 0, static_cast<cudaStream_t>(stream),
-             cache->k, cache->v, reinterpret_cast<__half*>(cache->ks), reinterpret_cast<__half*>(cache->vs),
-             reinterpret_cast<__half*>(cache->idx_key), pos0, k, v,
-             reinterpret_cast<const __half*>(idx_key));
-  if ((r = launched("cache_write_kernel"))) return r;
+  if ((r = launched("cache_write_kernel",
+                    launch_pdl(qsa::cache_write_kernel, dim3(n, QSA_HKV, 2), dim3(256), 0,
+                               static_cast<cudaStream_t>(stream), cache->k, cache->v,
+                               reinterpret_cast<__half*>(cache->ks), reinterpret_cast<__half*>(cache->vs),
+                               reinterpret_cast<__half*>(cache->idx_key), pos0, k, v,
+                               reinterpret_cast<const __half*>(idx_key)))))
+    return r;
   return ok();
 }
 
@@ -597,8 +605,12 @@ int qsa_device_status(int* status, void* stream) {
 int qsa_selftest_wait_timeout(void* stream) {
   int r = prepare_device();
   if (r) return r;
-  qsa::wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(device_status());
-  if ((r = launched("wait_selftest_kernel"))) return r;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(32);
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  if ((r = launched("wait_selftest_kernel", cudaLaunchKernelEx(&cfg, qsa::wait_selftest_kernel, device_status()))))
+    return r;
   return ok();
 }
 
