@@ -422,6 +422,14 @@ def test_decode_config2(gpu):
     _decode_case(gpu, synth.make_workload(2))
 
 
+@pytest.mark.parametrize("n", [1, 2, 4, 8])
+@pytest.mark.parametrize("pos0", [0, 1, 63, 64, 511, 512, 513, 2047, 2048, 2050, 8192, 30000])
+def test_decode_boundary_grid(gpu, pos0, n):
+    # n new cells after pos0 cached ones: token i sees pos0 + 1 + i cells, from a single cell to
+    # well past top_k = 2048 (the dense path up to 2048 visible cells, scores and selection beyond)
+    _decode_case(gpu, synth.make_workload(1, n=n, cells=pos0 + n), 0)
+
+
 def test_decode_small_ragged(gpu):
     wl = synth.make_workload(1, n=5, cells=2077)
     wl.top_k = 300
