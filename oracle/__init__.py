@@ -18,6 +18,8 @@ mlock + qsa_attn / qsa_merge decode tweaks" unless noted):
 * ``partials_row`` / ``merge_row`` -- split partials and their log-sum-exp
   merge (qsa_merge, section 2).
 * ``dense_attn_row`` -- brute-force softmax over every visible cell.
+* ``gate_row`` -- the output gate, O * sigmoid(gate) ("attention + gate",
+  section 3).
 * ``quantize`` / ``cache_write`` -- the int8 + per-32 fp16 scale quantizer.
 * ``rows`` -- the whole step for chosen rows of a call.
 
@@ -57,7 +59,8 @@ def configure(L):
     L.qsa_oracle_dense_attn_row.argtypes = [P, P, P, P, i64, P, dbl, P]
     L.qsa_oracle_quantize.argtypes = [P, i64, P, P]
     L.qsa_oracle_cache_write.argtypes = [P, P, P, P, P, i64, i32, P, P, P]
-    L.qsa_oracle_rows.argtypes = [P, P, P, P, P, i64, P, i32, P, P, P, i32, dbl, P, P, P, i64, i32]
+    L.qsa_oracle_gate_row.argtypes = [P, P]
+    L.qsa_oracle_rows.argtypes = [P, P, P, P, P, i64, P, i32, P, P, P, P, i32, dbl, P, P, P, i64, i32]
     return L
 
 
@@ -157,6 +160,15 @@ def dense_attn_row(cache, V: int, q: np.ndarray, scale: float) -> np.ndarray:
     return out
 
 
+def gate_row(out: np.ndarray, gate: np.ndarray) -> np.ndarray:
+    """out [24][256] times sigmoid(gate [24][256]) (a new array)."""
+    res = np.array(out, np.float64, copy=True, order="C")
+    g = np.ascontiguousarray(gate, np.float32)
+    assert res.shape == (24, 256) and g.shape == (24, 256)
+    lib().qsa_oracle_gate_row(_p(g), _p(res))
+    return res
+
+
 def quantize(x: np.ndarray):
     x = np.ascontiguousarray(x, np.float32).ravel()
     assert x.size % 32 == 0
@@ -178,8 +190,9 @@ def cache_write(cache, pos0: int, k: np.ndarray, v: np.ndarray, key: np.ndarray)
                                  pos0, n, _p(k), _p(v), _p(key))
 
 
-def rows(wl, row_ids=None, want_scores: bool = False, threads: int | None = None, top_k=None):
-    """Run the whole step for the given rows of workload ``wl`` (synth.Workload).
+def rows(wl, row_ids=None, want_scores: bool = False, threads: int | None = None, top_k=None, gate=None):
+    """Run the whole step for the given rows of workload ``wl`` (synth.Workload);
+    ``gate`` (float32 [wl.rows][24][256]) gates the outputs.
 
     Returns (out [nr][24][256] float64, ids [nr][top_k] int32, scores or None).
     """
@@ -199,6 +212,8 @@ def rows(wl, row_ids=None, want_scores: bool = False, threads: int | None = None
     ld = vis0 + int(row_ids.max()) if nr else 0
     scores = np.empty((nr, ld), np.float64) if want_scores else None
     threads = threads or (os.cpu_count() or 1)
-    lib().qsa_oracle_rows(*ptrs, _p(key), vis0, _p(row_ids), nr, _p(q), _p(iq), _p(iw), k, wl.scale,
+    g = None if gate is None else np.ascontiguousarray(gate, np.float32)
+    lib().qsa_oracle_rows(*ptrs, _p(key), vis0, _p(row_ids), nr, _p(q), _p(iq), _p(iw),
+                          None if g is None else _p(g), k, wl.scale,
                           _p(out), _p(ids), _p(scores) if scores is not None else None, ld, threads)
     return out, ids, scores

@@ -25,7 +25,14 @@
 //   4. split partials (m, l, o) over contiguous pieces of the selected list
 //      and their log-sum-exp merge M = max m_k, e_k = exp(m_k - M),
 //      L = sum l_k e_k, O = sum o_k e_k / L (qsa_merge, same page, section 2).
-//   5. the cache-write quantizer, per group of 32 fp32 values:
+//   5. the optional output gate, elementwise on the attention output:
+//        out = O * sigmoid(gate),  sigmoid(x) = 1 / (1 + exp(-x)),  gate fp32 [24][256]
+//      ("attention + gate" in "opus r20 track A ...", section 3; the gate rows
+//      travel with the query rows, Q plus gate making 12288 floats per token in
+//      "Round 5 Track C Report ...", section 1, Target 2).  The pages do not
+//      write the gate's function out; the logistic sigmoid is the plainest
+//      reading of a multiplicative output gate.
+//   6. the cache-write quantizer, per group of 32 fp32 values:
 //        amax = max |x|; s = fp16_rn(amax / 127 in fp32), saturated at 65504;
 //        q = clamp(rint(x / float(s)), -127, 127), all codes 0 when s == 0.
 //      The pages give only "int8 KV, fp16 scales"; the group of 32 and the
@@ -196,7 +203,12 @@ void merge_head(const double* m, const double* l, const double* o, int nsplit, i
     for (int d = 0; d < kD; ++d) out[d] /= L;
 }
 
-// Step 5 for one group of 32 values.
+// Step 5 for one row: out[24][256] multiplied by sigmoid(gate) elementwise.
+void gate_row(const float* gate, double* out) {
+  for (int i = 0; i < kHQ * kD; ++i) out[i] *= 1.0 / (1.0 + std::exp(-static_cast<double>(gate[i])));
+}
+
+// Step 6 for one group of 32 values.
 void quantize_group(const float* x, int8_t* q, uint16_t* scale_bits) {
   float amax = 0.0f;
   for (int i = 0; i < kGroup; ++i) amax = std::max(amax, std::fabs(x[i]));
@@ -215,10 +227,10 @@ void quantize_group(const float* x, int8_t* q, uint16_t* scale_bits) {
   }
 }
 
-// One full row: scores, selection, attention.  out [24][256]; ids [k];
-// scores_out (optional) [V].
-void row(const CacheView& c, int64_t V, const float* q, const uint16_t* iq, const float* iw, int k,
-         double scale, double* out, int32_t* ids, double* scores_out) {
+// One full row: scores, selection, attention, the gate when given.  out [24][256];
+// ids [k]; gate (optional) [24][256]; scores_out (optional) [V].
+void row(const CacheView& c, int64_t V, const float* q, const uint16_t* iq, const float* iw,
+         const float* gate, int k, double scale, double* out, int32_t* ids, double* scores_out) {
   std::vector<double> sc(static_cast<size_t>(V));
   index_scores(c.idx_key, V, iq, iw, sc.data());
   if (scores_out) std::copy(sc.begin(), sc.end(), scores_out);
@@ -226,6 +238,7 @@ void row(const CacheView& c, int64_t V, const float* q, const uint16_t* iq, cons
   for (int h = 0; h < kHQ; ++h)
     attn_head(c, q + static_cast<size_t>(h) * kD, h / kQPerKV, ids, k, scale,
               out + static_cast<size_t>(h) * kD);
+  if (gate) gate_row(gate, out);
 }
 
 }  // namespace
@@ -329,6 +342,9 @@ void qsa_oracle_dense_attn_row(const int8_t* k, const int8_t* v, const uint16_t*
   }
 }
 
+// The output gate of one row, in place: out [24][256] *= sigmoid(gate [24][256]).
+void qsa_oracle_gate_row(const float* gate, double* out) { gate_row(gate, out); }
+
 // Quantizer over ngroups groups of 32 values.
 void qsa_oracle_quantize(const float* x, int64_t ngroups, int8_t* q, uint16_t* scale_bits) {
   for (int64_t i = 0; i < ngroups; ++i) quantize_group(x + i * kGroup, q + i * kGroup, scale_bits + i);
@@ -354,18 +370,21 @@ void qsa_oracle_cache_write(int8_t* kc, int8_t* vc, uint16_t* ks, uint16_t* vs, 
 }
 
 // Rows rows[0..nrows) of one call; row r sees vis0 + r cells.  out [nrows][24][256],
-// ids [nrows][k], scores (optional) [nrows][vmax] with vmax = vis0 + max row.
-// Rows run in parallel over the host cores (independent by definition).
+// ids [nrows][k], gate (optional) [rows of the call][24][256], scores (optional)
+// [nrows][vmax] with vmax = vis0 + max row.  Rows run in parallel over the host
+// cores (independent by definition).
 void qsa_oracle_rows(const int8_t* k, const int8_t* v, const uint16_t* ks, const uint16_t* vs,
                      const uint16_t* idx_key, int64_t vis0, const int32_t* rows, int nrows,
-                     const float* q, const uint16_t* iq, const float* iw, int top_k, double scale,
-                     double* out, int32_t* ids, double* scores, int64_t ld_scores, int threads) {
+                     const float* q, const uint16_t* iq, const float* iw, const float* gate, int top_k,
+                     double scale, double* out, int32_t* ids, double* scores, int64_t ld_scores,
+                     int threads) {
   const CacheView c{k, v, ks, vs, idx_key};
 #pragma omp parallel for schedule(dynamic, 1) num_threads(threads > 0 ? threads : 1)
   for (int i = 0; i < nrows; ++i) {
     const int r = rows[i];
     row(c, vis0 + r, q + static_cast<size_t>(r) * kHQ * kD, iq + static_cast<size_t>(r) * kHI * kDI,
-        iw + static_cast<size_t>(r) * kHI, top_k, scale, out + static_cast<size_t>(i) * kHQ * kD,
+        iw + static_cast<size_t>(r) * kHI, gate ? gate + static_cast<size_t>(r) * kHQ * kD : nullptr,
+        top_k, scale, out + static_cast<size_t>(i) * kHQ * kD,
         ids + static_cast<size_t>(i) * top_k,
         scores ? scores + static_cast<size_t>(i) * ld_scores : nullptr);
   }

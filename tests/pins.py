@@ -332,6 +332,99 @@ def check_attn_order_and_padding():
     assert np.array_equal(oracle.attn_row(cache, q[0], padded, 1 / 16), base)
 
 
+def load_softmax_golden():
+    """The hand-worked softmax fixture: per-KV-head weights and V codes, the expected
+    outputs and the two-piece partials (tests/golden/attn_softmax_hand.txt)."""
+    vals, pieces = {}, {}
+    with open(os.path.join(GOLDEN, "attn_softmax_hand.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            head, body = [p.strip() for p in line.split("|", 1)]
+            if head.startswith("piece"):
+                g = int(head.split()[1][1:])
+                fields = [p.split() for p in line.split("|")[1:]]
+                pieces[g] = {f[0]: np.array([float(t) for t in f[1:]]) for f in fields}
+            else:
+                vals[head] = np.array([float(t) for t in body.split()])
+    return vals, pieces
+
+
+def softmax_golden_case():
+    """Cache, query and ids of the hand-worked softmax fixture (construction in the file)."""
+    vals, pieces = load_softmax_golden()
+    cache = synth.make_cache(81, 4)
+    cache.k[:] = 0
+    for c in range(4):
+        cache.k[c, :, c] = 1
+    cache.ks[:] = np.float16(1.0)
+    for g in range(2):
+        cache.v[:, g, :] = vals[f"a{g}"].astype(np.int8)[:, None]
+    cache.vs[:] = (2.0 ** -np.arange(8)).astype(np.float16)
+    q = np.zeros((24, 256), np.float32)
+    for h in range(24):
+        q[h, :4] = (16.0 * np.log(vals[f"w{h // 12}"])).astype(np.float32)
+    return cache, q, vals, pieces
+
+
+def check_attn_softmax_golden():
+    # logits ln w_c give softmax weights w_c / sum(w): pins the natural exp, the 1/16 scale
+    # applied to the dot product and the max subtraction, which the closed forms above
+    # (one cell, uniform, dominant) cannot tell apart
+    cache, q, vals, pieces = softmax_golden_case()
+    ids = np.arange(4, dtype=np.int32)
+    dims = 2.0 ** -(np.arange(256) // 32)
+    want = np.stack([vals["out"][h // 12] * dims for h in range(24)])
+    got = oracle.attn_row(cache, q, ids, 1 / 16)
+    assert np.allclose(got, want, rtol=1e-6, atol=0), (got[0, :2], got[12, :2])
+    # padding and order do not matter; the brute-force routine agrees
+    got2 = oracle.attn_row(cache, q, np.array([3, -1, 1, 0, 2], np.int32), 1 / 16)
+    assert np.allclose(got2, want, rtol=1e-6, atol=0)
+    assert np.allclose(oracle.dense_attn_row(cache, 4, q, 1 / 16), want, rtol=1e-6, atol=0)
+    # two pieces {0, 1}, {2, 3}: the hand-worked m, l and o of each
+    m, l, o = oracle.partials_row(cache, q, ids, 2, 1 / 16)
+    for h in range(24):
+        p = pieces[h // 12]
+        assert np.allclose(m[h], p["m"], rtol=0, atol=1e-6), (h, m[h])
+        assert np.allclose(l[h], p["l"], rtol=1e-6, atol=0), (h, l[h])
+        assert np.allclose(o[h], p["o"][:, None] * dims[None, :], rtol=1e-6, atol=1e-12), h
+    assert np.allclose(oracle.merge_row(m, l, o), want, rtol=1e-6, atol=0)
+
+
+def load_gate_golden():
+    vals = {}
+    with open(os.path.join(GOLDEN, "gate_hand.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            head, body = [p.strip() for p in line.split("|", 1)]
+            vals[head] = np.array([float(t) for t in body.split()])
+    return vals["gate"], vals["factor"]
+
+
+def check_gate_golden():
+    # out * sigmoid(g) at hand-worked points (1/2, 3/4, 1/4, 9/10, 1/10, 4/5, 1, ~0)
+    g, factor = load_gate_golden()
+    cache, q, vals, _ = softmax_golden_case()
+    ids = np.arange(4, dtype=np.int32)
+    idx = (np.arange(24)[:, None] + np.arange(256)[None, :]) % 8
+    gate = g[idx].astype(np.float32)
+    base = oracle.attn_row(cache, q, ids, 1 / 16)
+    dims = 2.0 ** -(np.arange(256) // 32)
+    want = np.stack([vals["out"][h // 12] * dims for h in range(24)]) * factor[idx]
+    got = oracle.gate_row(base, gate)
+    assert np.allclose(got, want, rtol=1e-6, atol=1e-20), (got[0, :4], want[0, :4])
+    assert abs(got[0, 1] - 22.5) <= 1e-5
+    # the whole step with the gate equals the ungated step times the gate
+    wl = synth.make_workload(0, cells=200)
+    wl.top_k = 64
+    gate2 = (synth.Stream(83, "gate").normal(wl.rows * 24 * 256) * 3).astype(np.float32).reshape(wl.rows, 24, 256)
+    plain, ids0, _ = oracle.rows(wl, threads=2)
+    gated, ids1, _ = oracle.rows(wl, threads=2, gate=gate2)
+    assert np.array_equal(ids0, ids1)
+    assert np.allclose(gated[0], plain[0] / (1.0 + np.exp(-gate2[0].astype(np.float64))), rtol=1e-14, atol=0)
+
+
 def check_dense_equivalence():
     # top_k >= visible: the whole step equals brute-force softmax over every visible cell
     wl = synth.make_workload(0, cells=96)
@@ -435,6 +528,6 @@ ALL_CHECKS = [
     check_quantize_patterns, check_cache_write_layout, check_index_score_golden,
     check_index_score_onehot, check_topk_bruteforce, check_topk_special, check_attn_single_cell,
     check_attn_uniform, check_attn_dominant, check_attn_gqa_and_groups,
-    check_attn_order_and_padding, check_dense_equivalence, check_merge_golden,
+    check_attn_order_and_padding, check_attn_softmax_golden, check_gate_golden, check_dense_equivalence, check_merge_golden,
     check_merge_split_invariance, check_causal_decode, check_causal_prefill,
 ]

@@ -33,17 +33,33 @@ MUTANTS = {
     "iq_transposed": ("half_to_double(iq[h * kDI + d])", "half_to_double(iq[d * kHI + h])"),
     "weight_index": ("static_cast<double>(iw[h]) * std::max", "static_cast<double>(iw[0]) * std::max"),
     "causal_off_by_one": ("row(c, vis0 + r, ", "row(c, vis0 + r + 1, "),
+    # the same slip made in all three softmax routines (attention, partials, brute force):
+    # every closed form and invariant still holds; only the hand-worked weights catch it
+    "softmax_exp2": [("std::exp(s[j] - m)", "std::exp2(s[j] - m)"), ("std::exp(s[c] - m)", "std::exp2(s[c] - m)")],
+    "logit_divided_by_scale": [("s.push_back(scale * dot);", "s.push_back(dot / scale);"),
+                               ("s[c] = scale * dot;", "s[c] = dot / scale;")],
+    "temperature_after_max": [("std::exp(s[j] - m)", "std::exp(0.5 * (s[j] - m))"),
+                              ("std::exp(s[c] - m)", "std::exp(0.5 * (s[c] - m))")],
+    "gate_sign": ("std::exp(-static_cast<double>(gate[i]))", "std::exp(static_cast<double>(gate[i]))"),
+    "gate_linear": ("out[i] *= 1.0 / (1.0 + std::exp(-static_cast<double>(gate[i])));",
+                    "out[i] *= static_cast<double>(gate[i]);"),
     "scale_dropped": ("s.push_back(scale * dot);\n    cells.push_back(ids[i]);\n  }\n  for (int d = 0; d < kD; ++d) out[d] = 0.0;",
                       "s.push_back(dot);\n    cells.push_back(ids[i]);\n  }\n  for (int d = 0; d < kD; ++d) out[d] = 0.0;"),
 }
 
 
-def _build_mutant(name, old, new, tmp):
+# mutants the hand-worked softmax weights must catch (the closed forms cannot)
+SOFTMAX_ONLY = {"softmax_exp2", "temperature_after_max", "logit_divided_by_scale"}
+
+
+def _build_mutant(name, edits, tmp):
     src = open(obuild.SRC).read()
-    assert src.count(old) >= 1, f"mutation site for {name} not found"
+    for old, new in edits:
+        assert src.count(old) >= 1, f"mutation site for {name} not found: {old!r}"
+        src = src.replace(old, new)
     path = os.path.join(tmp, f"{name}.cpp")
     with open(path, "w") as f:
-        f.write(src.replace(old, new))
+        f.write(src)
     lib = os.path.join(tmp, f"lib{name}.so")
     subprocess.run(["g++", "-std=c++17", "-O1", "-fPIC", "-shared", "-fopenmp", path, "-o", lib],
                    check=True)
@@ -52,10 +68,12 @@ def _build_mutant(name, old, new, tmp):
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_mutant_is_caught(name):
-    old, new = MUTANTS[name]
+    edits = MUTANTS[name]
+    if isinstance(edits, tuple):
+        edits = [edits]
     saved = oracle.lib()
     with tempfile.TemporaryDirectory() as tmp:
-        path = _build_mutant(name, old, new, tmp)
+        path = _build_mutant(name, edits, tmp)
         oracle._lib = oracle.configure(ctypes.CDLL(path))
         failed = []
         try:
@@ -67,3 +85,5 @@ def test_mutant_is_caught(name):
         finally:
             oracle._lib = saved
     assert failed, f"no pin caught mutant {name}"
+    if name in SOFTMAX_ONLY:
+        assert "check_attn_softmax_golden" in failed, failed
