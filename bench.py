@@ -1,19 +1,24 @@
 """Throughput of the QSA sparse-attention step on B200, one JSON line on rank 0.
 
-Default workload: decode at 64K cells -- every step appends n new cells
-(qsa_cache_write) and runs qsa_decode for n = 1, 2, ..., 8 draft tokens
-(36 tokens per step), top_k 2048, on synthetic inputs shaped like the model
-the pages describe.  ``--config`` picks another workload (0-4); prefill
-workloads report cells scored per second.
+Headline workload: decode at 64K cells -- every step runs qsa_decode for
+n = 1, 2, ..., 8 draft tokens (36 tokens per step), each call appending its
+n new cells itself, top_k 2048, on synthetic inputs shaped like the model the
+pages describe.  The line's ``configs`` object holds the other workloads of
+the metric, measured the same way: decode at 256K cells (64 splits) and the
+two prompt chunks (cells scored per second).  ``--config`` picks another
+headline workload (0-4), ``--configs`` the others.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--configs 2,3,4]
+                    [--impl reference]
 
-Timing: W untimed steps, then K steps between a barrier and a device
-synchronize on both sides, CUDA events on the launching stream, max over
-ranks.  Each step reads a different one of 4 copies of the cache, so every
-step's cache (80 MB at 64K cells) has left the 126 MB L2 since its last use.
-Multi-GPU runs are independent replicas (the step has no exchange):
-``value`` is the sum over ranks.
+Timing: W untimed steps, then passes of exactly K steps, each between a
+barrier and a device synchronize on both sides, CUDA events on the launching
+stream, repeated until --min-seconds of device time (so the clock sampler sees
+the GPU under load); the median pass counts, max over ranks.  Each step reads
+a different one of 4 copies of the cache, so every step's cache (80 MB at 64K
+cells) has left the 126 MB L2 since its last use.  Multi-GPU runs are
+independent replicas (the step has no exchange): ``value`` is the sum over
+ranks; ``--gpus N`` without torchrun around it starts the N ranks itself.
 """
 from __future__ import annotations
 
@@ -41,7 +46,10 @@ KERNEL_SOURCES = {
     "attn_kernel": "qsa_attn.cuh",
     "index_score_kernel": "qsa_index_score.cuh",
     "score_gemm_kernel": "qsa_score_gemm.cuh",
-    "topk": "qsa_topk_cluster.cuh",
+    "score_select_kernel": "qsa_prefill_select.cuh",
+    "prefill_final_kernel": "qsa_prefill_select.cuh",
+    "cluster_select_kernel+topk": "qsa_topk_cluster.cuh",
+    "cluster_select_kernel": "qsa_topk_cluster.cuh",
     "merge_kernel": "qsa_merge.cuh",
 }
 CELL_BYTES = 2 * 2 * 256 + 2 * 2 * 8 * 2      # K + V codes and their scales, both KV heads
@@ -55,8 +63,14 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", type=int, default=1, choices=range(5))
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--configs", default="2,3,4",
+                    help="more workloads measured into the line's `configs` object ('none' for none)")
+    ap.add_argument("--min-seconds", type=float, default=1.0,
+                    help="timed passes of --steps steps are repeated until this much device time")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    return ap.parse_args()
+    a = ap.parse_args()
+    a.configs = [] if a.configs in ("", "none") else [int(c) for c in a.configs.split(",")]
+    return a
 
 
 # ---------------------------------------------------------------- workloads
@@ -79,6 +93,7 @@ class Spec:
         else:
             self.T, self.pos0 = c["T"], c["pos0"]
             self.ns = [self.T]
+            self.nsplit = 0                               # the library's choice for T rows
             self.units = sum(self.pos0 + t + 1 for t in range(self.T))   # cells scored per step
             self.metric, self.unit = "prefill QSA cells-scored/s", "cells/s"
         self.name = synth.CONFIG_NAMES[cfg]
@@ -289,6 +304,162 @@ def run_reference(args, spec: Spec):
 
 # ---------------------------------------------------------------- CUDA leg
 
+def _packed(torch, arrays, device=None, pin=False):
+    """One contiguous byte buffer holding `arrays` (numpy), each piece 256-byte aligned;
+    returns (buffer, views in the arrays' dtypes and shapes)."""
+    offs, at = [], 0
+    for a in arrays:
+        offs.append(at)
+        at = (at + a.nbytes + 255) // 256 * 256
+    buf = torch.empty(max(at, 16), dtype=torch.uint8, device=device or "cpu")
+    if pin:
+        buf = buf.pin_memory()
+    views = []
+    for a, o in zip(arrays, offs):
+        v = buf[o:o + a.nbytes].view(getattr(torch, str(a.dtype))).view(*a.shape)
+        views.append(v)
+    return buf, views
+
+
+class Workload:
+    """Device state of one workload: rotating cache copies, packed step inputs, outputs."""
+
+    def __init__(self, torch, qsa, spec, dev):
+        self.spec = spec
+        wl, k_h, v_h, key_h = host_inputs(spec)
+        self.wl, self.k_h, self.v_h, self.key_h = wl, k_h, v_h, key_h
+        self.caches = [qsa.DeviceCache.from_host(wl.cache, dev) for _ in range(ROTATE)]
+        rows = max(spec.ns)
+        host = [np.ascontiguousarray(x) for x in (wl.q[:rows], wl.iq[:rows], wl.iw[:rows], k_h[:rows],
+                                                   v_h[:rows], key_h[:rows])]
+        self.h_buf, hv = _packed(torch, host, pin=True)
+        for view, a in zip(hv, host):
+            view.copy_(torch.from_numpy(a))
+        self.d_buf, (self.q, self.iq, self.iw, self.kn, self.vn, self.keyn) = _packed(torch, host, dev)
+        self.d_buf.copy_(self.h_buf)
+        self.out_rows = sum(spec.ns)
+        self.out = torch.empty(self.out_rows, 24, 256, dtype=torch.float32, device=dev)
+        self.out_h = torch.empty(self.out.shape, dtype=torch.float32).pin_memory()
+        if spec.kind == "decode":
+            nbytes = max(qsa.workspace_bytes(qsa.MODE_DECODE, n, spec.L, spec.top_k, spec.nsplit) for n in spec.ns)
+        else:
+            nbytes = qsa.workspace_bytes(qsa.MODE_PREFILL, spec.T, spec.pos0 + spec.T, spec.top_k)
+        self.ws = qsa.workspace(nbytes, dev)
+        # each call's views, made once (a caller with fixed buffers holds them)
+        self.calls, at = [], 0
+        for n in spec.ns:
+            self.calls.append((n, self.q[:n], self.iq[:n], self.iw[:n],
+                               (self.kn[:n], self.vn[:n], self.keyn[:n]), self.out[at:at + n]))
+            at += n
+        self.h2d_bytes = int(self.h_buf.numel())
+        self.d2h_bytes = int(self.out.numel() * 4)
+
+    def step(self, qsa, i):
+        """One step: every call of the workload through the public API, each appending
+        its rows' own cells in the same call (cache copy i % ROTATE)."""
+        spec, c = self.spec, self.caches[i % ROTATE]
+        for n, q, iq, iw, app, out in self.calls:
+            if spec.kind == "decode":
+                qsa.decode(c, spec.L, q, iq, iw, spec.top_k, spec.nsplit, self.wl.scale, ws=self.ws, out=out,
+                           append=app)
+            else:
+                qsa.prefill_chunk(c, spec.pos0, q, iq, iw, spec.top_k, self.wl.scale, ws=self.ws, out=out,
+                                  append=app)
+
+
+def measure(torch, qsa, spec, args, dev, stream, world, local, with_cpu):
+    """Device-resident rate (CUDA graphs of whole steps), end-to-end rate from pinned host
+    buffers, per-kernel times and the roofline of one workload."""
+    w = Workload(torch, qsa, spec, dev)
+    for i in range(args.warmup):
+        w.step(qsa, i)
+    torch.cuda.synchronize()
+
+    # ---- device-resident: each step captured once per cache copy in a CUDA graph
+    graphs, per_graph = [], 0
+    for r in range(ROTATE):
+        g = torch.cuda.CUDAGraph()
+        before = qsa.launch_count()
+        with torch.cuda.graph(g):
+            w.step(qsa, r)
+        per_graph = qsa.launch_count() - before
+        graphs.append(g)
+    for i in range(max(args.warmup, ROTATE)):
+        graphs[i % ROTATE].replay()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def timed_pass(k, fn):
+        barrier(world)
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for i in range(k):
+            fn(i)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        return ev0.elapsed_time(ev1)
+
+    replay = lambda i: graphs[i % ROTATE].replay()  # noqa: E731
+    if args.steps:
+        steps = args.steps
+    else:  # about a quarter second per pass
+        per_step = timed_pass(2 * ROTATE, replay) / (2 * ROTATE)
+        steps = int(dist_max(float(max(20, min(100000, 250.0 / max(per_step, 1e-3)))), world))
+    # Passes of exactly `steps` steps until at least min_seconds of timed work, so the clock
+    # sampler sees the GPU under load; the median pass is reported.
+    first = timed_pass(steps, replay)
+    passes = int(dist_max(float(max(3, min(10000, -(-args.min_seconds * 1000.0 // max(first, 1e-3))))), world))
+    with ClockSampler(local) as clk:
+        times = [timed_pass(steps, replay) for _ in range(passes)]
+    ms_pass = statistics.median(times)
+    value, ms_max = job_rate(spec.units, steps, ms_pass, world)
+    for g in graphs:
+        g.reset()
+    del graphs
+
+    # ---- end to end through the public API: one copy of the packed inputs from pinned host
+    # memory, the calls (each appending its rows' cells), one copy of all outputs back
+    def e2e_step(i):
+        w.d_buf.copy_(w.h_buf, non_blocking=True)
+        w.step(qsa, i)
+        w.out_h.copy_(w.out, non_blocking=True)
+
+    for i in range(2):
+        e2e_step(i)
+    e2e_times = [timed_pass(steps, e2e_step) for _ in range(3)]
+    e2e_value, _ = job_rate(spec.units, steps, statistics.median(e2e_times), world)
+
+    # ---- per-kernel durations, step-level calls with events on the same stream
+    kern = kernel_times(qsa, torch, w, spec, stream, 20)
+    roof = roofline(spec, kern, peaks())
+    res = {"metric": spec.metric, "value": value, "unit": spec.unit, "ms_per_step": ms_max / steps,
+           "steps": steps, "passes": passes,
+           "config": {"workload": spec.name, "cells": spec.L, "top_k": spec.top_k,
+                      "rows_per_call": spec.ns if spec.kind == "decode" else spec.T,
+                      "nsplit": spec.nsplit if spec.kind == "decode" else "auto",
+                      "l2": f"{ROTATE} rotating cache copies "
+                            f"({ROTATE * spec.L * (CELL_BYTES + KEY_BYTES) / 1e6:.0f} MB > 126 MB L2)",
+                      "timing": f"median of {passes} passes of {steps} graph-replayed steps"},
+           "e2e": {"value": e2e_value, "unit": spec.unit, "h2d_bytes_per_step": w.h2d_bytes,
+                   "d2h_bytes_per_step": w.d2h_bytes,
+                   "api": "one H2D copy of the packed inputs, one call per row group appending its "
+                          "cells (qsa_decode / qsa_prefill_chunk with append), one D2H copy of the outputs"},
+           "gpu_launches": per_graph * steps,
+           "roofline": roof["main"], "kernels": roof["kernels"], "clocks": clk.summary()}
+    if "score_attn" in roof:
+        res["roofline_score_attn"] = roof["score_attn"]
+    if "score_gemm" in roof:
+        res["roofline_score_gemm"] = roof["score_gemm"]
+    if with_cpu:
+        val, cores, what, dt = oracle_sample(spec, w.wl, w.k_h, w.v_h, w.key_h, 15.0)
+        res["cpu_baseline"] = {"value": val, "unit": spec.unit, "cores": cores, "kind": "oracle",
+                               "sample": f"{what}, {dt:.1f} s"}
+    del w
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_cuda(args, spec: Spec):
     import torch
 
@@ -304,149 +475,27 @@ def run_cuda(args, spec: Spec):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
 
-    wl, k_h, v_h, key_h = host_inputs(spec)
-    caches = [qsa.DeviceCache.from_host(wl.cache, dev) for _ in range(ROTATE)]
-    q = torch.from_numpy(wl.q).to(dev)
-    iq = torch.from_numpy(wl.iq).to(dev)
-    iw = torch.from_numpy(wl.iw).to(dev)
-    kn = torch.from_numpy(k_h).to(dev)
-    vn = torch.from_numpy(v_h).to(dev)
-    keyn = torch.from_numpy(key_h).to(dev)
-    nmax = max(spec.ns)
-    if spec.kind == "decode":
-        ws_bytes = max(qsa.workspace_bytes(qsa.MODE_DECODE, n, spec.L, spec.top_k, spec.nsplit)
-                       for n in spec.ns)
-    else:
-        ws_bytes = qsa.workspace_bytes(qsa.MODE_PREFILL, spec.T, spec.pos0 + spec.T, spec.top_k)
-    ws = qsa.workspace(ws_bytes, dev)
-    out = torch.empty(nmax, 24, 256, dtype=torch.float32, device=dev)
-    ids = torch.empty(nmax, spec.top_k, dtype=torch.int32, device=dev)
+    head = measure(torch, qsa, spec, args, dev, stream, world, local,
+                   with_cpu=rank == 0 and world == 1 and not args.no_cpu_baseline)
+    extra = {}
+    for cfg in args.configs:
+        if cfg == spec.cfg:
+            continue
+        sub = measure(torch, qsa, Spec(cfg), args, dev, stream, world, local, with_cpu=False)
+        extra[sub["config"]["workload"]] = sub
 
-    def step(i, qq=q, iqq=iq, iww=iw, kk=kn, vv=vn, key=keyn, o=out):
-        c = caches[i % ROTATE]
-        for n in spec.ns:
-            if spec.kind == "decode":
-                qsa.cache_write(c, spec.L - n, kk[:n], vv[:n], key[:n])
-                qsa.decode(c, spec.L, qq[:n], iqq[:n], iww[:n], spec.top_k, spec.nsplit, wl.scale,
-                           ws=ws, out=o[:n], ids_out=ids[:n])
-            else:
-                qsa.cache_write(c, spec.pos0, kk, vv, key)
-                qsa.prefill_chunk(c, spec.pos0, qq, iqq, iww, spec.top_k, wl.scale, ws=ws, out=o,
-                                  ids_out=ids)
-
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize()
-
-    # ---- device-resident throughput: each step (all its calls) captured once per cache copy
-    # in a CUDA graph, so the timed loop measures the kernels, not Python's launch overhead
-    graphs, per_graph = [], 0
-    for r in range(ROTATE):
-        g = torch.cuda.CUDAGraph()
-        before = qsa.launch_count()
-        with torch.cuda.graph(g):
-            step(r)
-        per_graph = qsa.launch_count() - before
-        graphs.append(g)
-    for i in range(args.warmup):
-        graphs[i % ROTATE].replay()
-    torch.cuda.synchronize()
-    if args.steps:
-        steps = args.steps
-    else:  # about two seconds of timed work, so the clock sampler sees the GPU under load
-        probe0, probe1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        probe0.record(stream)
-        for i in range(2 * ROTATE):
-            graphs[i % ROTATE].replay()
-        probe1.record(stream)
-        torch.cuda.synchronize()
-        per_step = probe0.elapsed_time(probe1) / (2 * ROTATE)
-        steps = int(max(20, min(100000, 2000.0 / max(per_step, 1e-3))))
-        steps = int(dist_max(float(steps), world))
-    barrier(world)
-    torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
-        ev0.record(stream)
-        for i in range(steps):
-            graphs[i % ROTATE].replay()
-        ev1.record(stream)
-        torch.cuda.synchronize()
-    launches = per_graph * steps
-    ms = ev0.elapsed_time(ev1)
-    barrier(world)
-    value, ms_max = job_rate(spec.units, steps, ms, world)
-
-    # ---- end to end through the public API from pinned host buffers
-    q_h = torch.from_numpy(wl.q).pin_memory()
-    iq_h = torch.from_numpy(wl.iq).pin_memory()
-    iw_h = torch.from_numpy(wl.iw).pin_memory()
-    kk_h = torch.from_numpy(k_h).pin_memory()
-    vv_h = torch.from_numpy(v_h).pin_memory()
-    key_hh = torch.from_numpy(key_h).pin_memory()
-    out_h = torch.empty(out.shape, dtype=torch.float32).pin_memory()
-    qd, iqd, iwd = torch.empty_like(q), torch.empty_like(iq), torch.empty_like(iw)
-    kd, vd, keyd = torch.empty_like(kn), torch.empty_like(vn), torch.empty_like(keyn)
-    h2d = sum(t.numel() * t.element_size() for t in (q_h, iq_h, iw_h, kk_h, vv_h, key_hh))
-    d2h = 0
-    for n in spec.ns:
-        d2h += n * 24 * 256 * 4
-
-    # each call's row views, made once (a caller with fixed buffers holds them)
-    views = {n: (kd[:n], vd[:n], keyd[:n], qd[:n], iqd[:n], iwd[:n], out[:n], out_h[:n]) for n in spec.ns}
-
-    def e2e_step(i):
-        for dst, src in ((qd, q_h), (iqd, iq_h), (iwd, iw_h), (kd, kk_h), (vd, vv_h), (keyd, key_hh)):
-            dst.copy_(src, non_blocking=True)
-        c = caches[i % ROTATE]
-        for n in spec.ns:
-            if spec.kind == "decode":
-                kn_, vn_, keyn_, qn_, iqn_, iwn_, outn_, outhn_ = views[n]
-                qsa.cache_write(c, spec.L - n, kn_, vn_, keyn_)
-                qsa.decode(c, spec.L, qn_, iqn_, iwn_, spec.top_k, spec.nsplit, wl.scale, ws=ws, out=outn_)
-                outhn_.copy_(outn_, non_blocking=True)
-            else:
-                qsa.cache_write(c, spec.pos0, kd, vd, keyd)
-                qsa.prefill_chunk(c, spec.pos0, qd, iqd, iwd, spec.top_k, wl.scale, ws=ws, out=out)
-                out_h.copy_(out, non_blocking=True)
-
-    for i in range(2):
-        e2e_step(i)
-    barrier(world)
-    torch.cuda.synchronize()
-    ev0.record(stream)
-    for i in range(steps):
-        e2e_step(i)
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    e2e_value, _ = job_rate(spec.units, steps, ev0.elapsed_time(ev1), world)
-
-    # ---- per-kernel durations, step-level calls with events on the same stream
-    kern = kernel_times(qsa, torch, spec, caches, wl, q, iq, iw, ws, dev, stream, 20)
-    pk = peaks()
-    roof = roofline(spec, kern, pk)
-
-    line = {"metric": spec.metric, "value": value, "unit": spec.unit, "n_gpus": world, "steps": steps,
-            "warmup": args.warmup, "ms_per_step": ms_max / steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-            "config": {"workload": spec.name, "cells": spec.L, "top_k": spec.top_k,
-                       "rows_per_call": spec.ns if spec.kind == "decode" else spec.T,
-                       "nsplit": spec.nsplit if spec.kind == "decode" else "auto",
-                       "l2": f"{ROTATE} rotating cache copies "
-                             f"({ROTATE * spec.L * (CELL_BYTES + KEY_BYTES) / 1e6:.0f} MB > 126 MB L2)",
-                       "parallelism": "replicas" if world > 1 else "single GPU"},
-            "e2e": {"value": e2e_value, "unit": spec.unit, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches,
-            "roofline": roof["main"],
-            "kernels": roof["kernels"],
-            "clocks": clk.summary()}
-    if spec.kind == "decode" and "score_attn" in roof:
-        line["roofline_score_attn"] = roof["score_attn"]
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        val, cores, what, dt = oracle_sample(spec, wl, k_h, v_h, key_h, 15.0)
-        line["cpu_baseline"] = {"value": val, "unit": spec.unit, "cores": cores, "kind": "oracle",
-                                "sample": f"{what}, {dt:.1f} s"}
+    line = {"metric": head["metric"], "value": head["value"], "unit": head["unit"], "n_gpus": world,
+            "steps": head["steps"], "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+            "data": "synthetic", "config": dict(head["config"],
+                                                parallelism="replicas" if world > 1 else "single GPU"),
+            "e2e": head["e2e"], "gpu_launches": head["gpu_launches"], "roofline": head["roofline"],
+            "kernels": head["kernels"], "clocks": head["clocks"]}
+    for key in ("roofline_score_attn", "roofline_score_gemm", "cpu_baseline"):
+        if key in head:
+            line[key] = head[key]
+    if extra:
+        line["configs"] = extra
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -454,62 +503,43 @@ def run_cuda(args, spec: Spec):
         dist.destroy_process_group()
 
 
-def kernel_times(qsa, torch, spec, caches, wl, q, iq, iw, ws, dev, stream, reps):
-    """Average duration of each step kernel, from CUDA events around the
-    step-level calls (the same kernels qsa_decode / qsa_prefill_chunk launch)."""
-    acc = {"index_score_kernel": 0.0, "topk": 0.0, "attn_kernel": 0.0, "merge_kernel": 0.0}
-    count = {k: 0 for k in acc}
-    info = {"union_cells": 0, "rows": 0, "cells_scored": 0, "ncells": 0, "nsplit": {}}
-    ld_max = (spec.L + 3) // 4 * 4
-    nmax = max(spec.ns)
-    scores = torch.empty(nmax, ld_max, dtype=torch.float32, device=dev)
-    tk_ws = qsa.workspace(qsa.topk_workspace_bytes(nmax, spec.L, spec.top_k), dev)
-    ids = torch.empty(nmax, spec.top_k, dtype=torch.int32, device=dev)
-    out = torch.empty(nmax, 24, 256, dtype=torch.float32, device=dev)
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
-    parts = {}
-    # Each call sits behind a ~1.5 ms torch sleep kernel so the host has queued all of
-    # its launches before the first starts: the events bracket kernels, not launch gaps.
+def kernel_times(qsa, torch, w, spec, stream, reps):
+    """Average device time of every kernel the step's calls launch, per launch, from the
+    library's own trace events (qsa_trace_begin / qsa_trace_end) around the real calls."""
+    acc, count = {}, {}
+    info = {"union_cells": 0, "rows": 0, "cells_scored": 0, "ncells": 0, "nsplit": {}, "calls": 0}
+    ids = torch.empty(max(spec.ns), spec.top_k, dtype=torch.int32, device=w.out.device)
+    # Each call sits behind a ~1.5 ms torch sleep kernel so the host has queued all of its
+    # launches before the first starts: the events bracket kernels, not launch gaps.
     for rep in range(reps + 2):
-        c = caches[rep % ROTATE]
-        for n in spec.ns:
-            if spec.kind == "decode":
-                vis0, ncells = spec.L - n + 1, spec.L
-                ns = spec.nsplit or auto_nsplit(n, spec.top_k)
-            else:
-                vis0, ncells = spec.pos0 + 1, spec.pos0 + spec.T
-                ns = auto_nsplit(n, spec.top_k)
-            part = parts.setdefault((n, ns), torch.empty(n, 24, ns, 258, dtype=torch.float32, device=dev)
-                                  if ns > 1 else None)
+        c = w.caches[rep % ROTATE]
+        for n, q, iq, iw, app, out in w.calls:
             torch.cuda._sleep(3_000_000)
-            ev[0].record(stream)
-            qsa.index_score(c, iq[:n], iw[:n], ncells, scores=scores[:n])
-            ev[1].record(stream)
-            qsa.topk(scores[:n], vis0, spec.top_k, ws=tk_ws, ids=ids[:n])
-            ev[2].record(stream)
-            res = qsa.attn(c, q[:n], ids[:n], ns, wl.scale, part=part, out=out[:n] if ns == 1 else None)
-            ev[3].record(stream)
-            if ns > 1:
-                qsa.merge(res, out=out[:n])
-            ev[4].record(stream)
-            torch.cuda.synchronize()
+            with qsa.trace(stream=torch.cuda.current_stream()) as tr:
+                if spec.kind == "decode":
+                    qsa.decode(c, spec.L, q, iq, iw, spec.top_k, spec.nsplit, w.wl.scale, ws=w.ws, out=out,
+                               ids_out=ids[:n], append=app)
+                else:
+                    qsa.prefill_chunk(c, spec.pos0, q, iq, iw, spec.top_k, w.wl.scale, ws=w.ws, out=out,
+                                      ids_out=ids[:n], append=app)
             if rep < 2:
                 continue
-            names = list(acc)
-            for j in range(4):
-                if j == 3 and ns == 1:
-                    continue
-                acc[names[j]] += ev[j].elapsed_time(ev[j + 1])
-                count[names[j]] += 1
+            for name, ms in tr.kernels:
+                acc[name] = acc.get(name, 0.0) + ms
+                count[name] = count.get(name, 0) + 1
             if rep == 2:
+                vis0 = spec.L - n + 1 if spec.kind == "decode" else spec.pos0 + 1
+                ncells = spec.L if spec.kind == "decode" else spec.pos0 + spec.T
                 idn = ids[:n].cpu().numpy()
                 info["union_cells"] += int(np.unique(idn[idn >= 0]).size)
                 info["rows"] += n
                 info["cells_scored"] += int(sum(vis0 + r for r in range(n)))
                 info["ncells"] += ncells * n
-                info["nsplit"][n] = ns
-    avg = {k: (acc[k] / count[k] if count[k] else None) for k in acc}
-    return {"avg_ms": avg, "launches": count, "info": info, "reps": reps}
+                info["nsplit"][n] = spec.nsplit or auto_nsplit(n, spec.top_k)
+                info["calls"] += 1
+    avg = {k: acc[k] / count[k] for k in acc}
+    per_call = {k: count[k] / (reps * len(spec.ns)) for k in acc}  # launches of each kernel per call
+    return {"avg_ms": avg, "launches_per_call": per_call, "info": info, "reps": reps}
 
 
 def auto_nsplit(rows, top_k):
@@ -519,67 +549,84 @@ def auto_nsplit(rows, top_k):
     return max(1, min(64, max(1, top_k // 32), want))
 
 
+SELECTION_KERNELS = ("cluster_select_kernel", "topk_zero_kernel", "topk_hist_kernel", "topk_filter_kernel",
+                     "topk_final_kernel")
+
+
 def roofline(spec, kern, pk):
-    """Algorithmic bytes (or flops) per launch over measured launch time, for
-    every step kernel; the dominant one (most time per call) is `main`."""
-    info, avg = kern["info"], kern["avg_ms"]
-    calls = len(spec.ns)
+    """Algorithmic bytes (or flops) per launch over measured launch time, for every step
+    kernel; the dominant one (most time per call) is `main`."""
+    info, avg, per_call = kern["info"], kern["avg_ms"], kern["launches_per_call"]
+    calls = max(1, info["calls"])
     hbm, tensor = pk["hbm_gbs"], pk["bf16_tflops"]
     rows = info["rows"] / calls
     ncells = info["ncells"] / calls                      # (row, cell) scores per call
+    cells_scored = info["cells_scored"] / calls          # visible (row, cell) pairs per call
     kernels = {}
 
     def hbm_entry(name, nbytes, note):
-        ms = avg[name]
+        ms = avg.get(name)
         if not ms:
-            return None
+            return
         ach = nbytes / (ms / 1e3) / 1e9
-        return {"kernel": name, "bound": "hbm", "ms": ms, "bytes_per_launch": nbytes, "achieved": ach,
-                "peak": hbm, "unit": "GB/s", "frac": ach / hbm, "note": note}
+        kernels[name] = {"kernel": name, "bound": "hbm", "ms": ms, "bytes_per_launch": nbytes, "achieved": ach,
+                         "peak": hbm, "unit": "GB/s", "frac": ach / hbm, "note": note}
 
-    # index score: keys once, scores written once (decode); prefill: 512 flops per visible cell
     key_bytes = spec.L * KEY_BYTES
-    if spec.kind == "decode":
-        kernels["index_score_kernel"] = hbm_entry("index_score_kernel", key_bytes + 4 * ncells,
-                                                  "keys read once + fp32 scores written")
-    else:
-        ms = avg["index_score_kernel"]
-        flops = 512.0 * info["cells_scored"] / calls
-        ach = flops / (ms / 1e3) / 1e12
-        kernels["index_score_kernel"] = {"kernel": "score_gemm_kernel (tcgen05)", "bound": "tensor", "ms": ms,
-                                         "flops_per_launch": flops, "achieved": ach, "peak": tensor,
-                                         "unit": "TFLOP/s", "frac": ach / tensor,
-                                         "note": "512 flops per visible (row, cell); fp16 has bf16's nominal rate"}
-    # selection: every visible score read, ids written
-    kernels["topk"] = hbm_entry("topk", 4 * info["cells_scored"] / calls + 4 * rows * spec.top_k,
-                                "visible scores read + ids written (decode: one cluster kernel; "
-                                "prefill: histogram, filter and final kernels together)")
-    # attention: the union of the rows' selected cells (K, V, scales) + queries, ids, outputs
     attn_bytes = (info["union_cells"] * CELL_BYTES + info["rows"] * (24 * 256 * 4 * 2 + spec.top_k * 4)) / calls
-    kernels["attn_kernel"] = hbm_entry("attn_kernel", attn_bytes,
-                                       "union of the rows' selected cells x 1088 B + q, ids, out"
-                                       + (" (prefill: gathered from L2 mostly)" if spec.kind == "prefill" else ""))
-    if avg["merge_kernel"]:
+    hbm_entry("index_score_kernel", key_bytes + 4 * ncells,
+              "keys read once + fp32 scores written (the call's new cells quantized in the same launch)")
+    sel = [k for k in SELECTION_KERNELS if k in avg]
+    if sel:  # the decode selection: one cluster kernel, or the multi-kernel path for long rows
+        ms = sum(avg[k] * per_call[k] for k in sel)
+        nbytes = 4 * cells_scored + 4 * rows * spec.top_k
+        ach = nbytes / (ms / 1e3) / 1e9
+        kernels["selection"] = {"kernel": "+".join(sel), "bound": "hbm", "ms": ms, "bytes_per_launch": nbytes,
+                                "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                                "note": "visible scores read + ids written"}
+    if "score_select_kernel" in avg:
+        ms = avg["score_select_kernel"]
+        flops = 512.0 * cells_scored
+        ach = flops / (ms / 1e3) / 1e12
+        kernels["score_select_kernel"] = {
+            "kernel": "score_select_kernel (tcgen05)", "bound": "tensor", "ms": ms, "flops_per_launch": flops,
+            "achieved": ach, "peak": tensor, "unit": "TFLOP/s", "frac": ach / tensor,
+            "note": "512 flops per visible (row, cell); fp16 has bf16's nominal rate; candidates only written"}
+    hbm_entry("prefill_threshold_kernel", key_bytes / 16 + 16 * rows,
+              "every 16th key (the sample) + thresholds; the sampled keys are re-read from L2 per 8 rows")
+    hbm_entry("prefill_final_kernel", 4 * rows * spec.top_k,
+              "ids written (the candidate lists are read from L2)")
+    hbm_entry("cache_write_kernel", rows * (2 * 2 * 256 * 4 + 128 + CELL_BYTES + KEY_BYTES),
+              "new cells: fp32 K/V and fp16 keys read, int8 codes, fp16 scales and keys written")
+    hbm_entry("attn_kernel", attn_bytes, "union of the rows' selected cells x 1088 B + q, ids, out"
+              + (" (prefill: gathered from L2 mostly)" if spec.kind == "prefill" else ""))
+    if "merge_kernel" in avg:
         ns = info["nsplit"]
         part_bytes = sum(n * 24 * ns[n] * 258 * 4 + n * 24 * 256 * 4 for n in ns) / calls
-        kernels["merge_kernel"] = hbm_entry("merge_kernel", part_bytes, "partials read + output written")
-    kernels = {k: v for k, v in kernels.items() if v}
-    dom = max(kernels, key=lambda k: kernels[k]["ms"] or 0)
+        hbm_entry("merge_kernel", part_bytes, "partials read + output written")
+    # per call: a kernel's time times its launches per call
+    for k, v in kernels.items():
+        v["ms_per_call"] = v["ms"] * (1 if k == "selection" else per_call.get(k, 1))
+    dom = max(kernels, key=lambda k: kernels[k]["ms_per_call"])
     main = dict(kernels[dom])
     main["peak_source"] = pk["source"]
-    main["traffic"] = traffic_for(dom, spec.name)
+    main["traffic"] = traffic_for(main["kernel"].split(" ")[0], spec.name)
     out = {"kernels": kernels, "main": main}
-    if spec.kind == "decode":
+    if spec.kind == "decode" and "index_score_kernel" in avg and "attn_kernel" in avg:
         both_b = key_bytes + attn_bytes
         both_t = (avg["index_score_kernel"] + avg["attn_kernel"]) / 1e3
         out["score_attn"] = {"bound": "hbm", "achieved": both_b / both_t / 1e9, "peak": hbm, "unit": "GB/s",
                              "frac": both_b / both_t / 1e9 / hbm,
                              "note": "keys + union of selected cells over the two kernels' summed time"}
+    if "score_select_kernel" in kernels:
+        out["score_gemm"] = dict(kernels["score_select_kernel"], peak_source=pk["source"])
     return out
 
 
 def main():
     args = parse()
+    if args.gpus > 1 and "RANK" not in os.environ:
+        sys.exit(relaunch(args))
     spec = Spec(args.config)
     if args.impl == "reference":
         run_reference(args, spec)

@@ -58,6 +58,7 @@ extern "C" {
 #define QSA_MAX_SPLITS 64   /* context splits merged by log-sum-exp */
 #define QSA_MAX_TOPK 16384  /* largest top_k */
 #define QSA_MAX_CELLS (1 << 24)
+#define QSA_MAX_ROWS 65535  /* query rows of one prefill, qsa_topk or qsa_attn call */
 #define QSA_PART_STRIDE (2 + QSA_D) /* floats per partial: m, l, o[256] */
 
 enum {
@@ -89,6 +90,24 @@ typedef struct qsa_cache {
 } qsa_cache;
 
 /*
+ * The call's own new cells (the write side of qsa_prep: "Round 5 Track C
+ * Report ...", section 1, Targets 1-2, kcur / vcur rows of 2 x 256 floats per
+ * token), appended by the step call itself before anything reads the cache:
+ * qsa_decode writes its n tokens' cells at L - n .. L - 1, qsa_prefill_chunk
+ * its T tokens' cells at pos0 .. pos0 + T - 1, exactly as qsa_cache_write
+ * would (same quantizer, bit for bit).  One call then does what a cache
+ * write followed by a step does, with one host crossing.  Caller-owned device
+ * memory:
+ *   k, v     fp32 [rows][2][256]
+ *   idx_key  fp16 [rows][64]
+ */
+typedef struct qsa_new_cells {
+  const float* k;
+  const float* v;
+  const uint16_t* idx_key;
+} qsa_new_cells;
+
+/*
  * Bytes of workspace qsa_decode (mode QSA_MODE_DECODE, rows = n, L = cache
  * length) or qsa_prefill_chunk (mode QSA_MODE_PREFILL, rows = T, L = pos0 + T)
  * needs for these sizes; nsplit as passed to the call (0 = automatic).
@@ -112,9 +131,16 @@ int qsa_cache_write(const qsa_cache* cache, int pos0, int n, const float* k, con
 /*
  * Decode step for n = 1..8 query tokens (the MTP draft of "opus r20 track A
  * ...", section 3, ntok 1..8).  Token i sees cells [0, L - n + 1 + i).
- *   q   fp32 [n][24][256]     query rows
- *   iq  fp16 [n][4][64]       indexer queries
- *   iw  fp32 [n][4]           indexer head weights
+ *   append  the n tokens' own cells, written at L - n .. L - 1 first (see
+ *           qsa_new_cells), or NULL when they are already in the cache
+ *   q       fp32 [n][24][256]     query rows
+ *   iq      fp16 [n][4][64]       indexer queries
+ *   iw      fp32 [n][4]           indexer head weights
+ *   gate    fp32 [n][24][256] or NULL: the output gate ("attention + gate",
+ *           same page, section 3; the gate rows travel with the query rows,
+ *           12288 floats per token of Q plus gate in "Round 5 Track C Report
+ *           ...", section 1, Target 2): out = O * sigmoid(gate), elementwise,
+ *           sigmoid(x) = 1 / (1 + exp(-x)); NULL leaves O ungated
  * Per token: score[c] = sum_h iw[h] * max(0, iq[h] . idx_key[c]) for every
  * visible c; the top_k cells of largest score (equal scores: lower index
  * first; all visible cells when fewer than top_k); then for head h
@@ -132,23 +158,28 @@ int qsa_cache_write(const qsa_cache* cache, int pos0, int n, const float* k, con
  * Requires 1 <= n <= 8, n <= L <= max_cells, 1 <= top_k <= QSA_MAX_TOPK,
  * 0 <= nsplit <= QSA_MAX_SPLITS.
  */
-int qsa_decode(const qsa_cache* cache, int L, int n, const float* q, const uint16_t* iq,
-               const float* iw, int top_k, int nsplit, float scale, void* ws, size_t ws_bytes,
-               float* out, int32_t* ids_out, void* stream);
+int qsa_decode(const qsa_cache* cache, int L, int n, const qsa_new_cells* append, const float* q,
+               const uint16_t* iq, const float* iw, const float* gate, int top_k, int nsplit,
+               float scale, void* ws, size_t ws_bytes, float* out, int32_t* ids_out, void* stream);
 
 /*
  * Prefill step for a causal chunk of T tokens at pos0 (prompt_chunk with
  * qsa_score_mm, qsa_topk and the prompt attention: "opus r15 track A ...",
  * what changed, items 1-2; "Round 5 Track C Report ...", section 2.1).  Row t
- * sees cells [0, pos0 + t]; the chunk's own cells must already be written.
- * Arguments as qsa_decode with n -> T (q [T][24][256], iq [T][4][64],
- * iw [T][4], out [T][24][256], ids_out [T][top_k] or NULL).  A chunk with
- * pos0 + T <= top_k takes the dense path, as qsa_decode does.
- * Requires 0 <= pos0, 1 <= T, pos0 + T <= max_cells.
+ * sees cells [0, pos0 + t]; the chunk's own cells are written first from
+ * `append`, or must already be in the cache when `append` is NULL.
+ * Arguments as qsa_decode with n -> T (append rows [T], q [T][24][256],
+ * iq [T][4][64], iw [T][4], gate [T][24][256] or NULL, out [T][24][256],
+ * ids_out [T][top_k] or NULL).  A chunk with pos0 + T <= top_k takes the dense
+ * path, as qsa_decode does.  The score GEMM of a chunk waits on mbarriers
+ * (bounded): after the results are used, a caller that must know they are
+ * sound checks qsa_device_status once.
+ * Requires 0 <= pos0, 1 <= T <= QSA_MAX_ROWS, pos0 + T <= max_cells.
  */
-int qsa_prefill_chunk(const qsa_cache* cache, int pos0, int T, const float* q,
-                      const uint16_t* iq, const float* iw, int top_k, float scale, void* ws,
-                      size_t ws_bytes, float* out, int32_t* ids_out, void* stream);
+int qsa_prefill_chunk(const qsa_cache* cache, int pos0, int T, const qsa_new_cells* append,
+                      const float* q, const uint16_t* iq, const float* iw, const float* gate,
+                      int top_k, float scale, void* ws, size_t ws_bytes, float* out,
+                      int32_t* ids_out, void* stream);
 
 /* ---- the four steps, one call each (used by the composite calls above) ---- */
 
@@ -157,6 +188,8 @@ int qsa_prefill_chunk(const qsa_cache* cache, int pos0, int T, const float* q,
  * scores[r * ld + c] = sum_h iw[r][h] * max(0, sum_d iq[r][h][d] * idx_key[c][d])
  * for rows r < rows and cells c < ncells (fp16 products, fp32 accumulation).
  * Callers mask by visibility.  ld >= ncells, ld % 4 == 0, ncells <= max_cells.
+ * More than 8 rows run the tcgen05 GEMM, whose bounded waits report through
+ * qsa_device_status.
  */
 int qsa_index_score(const qsa_cache* cache, int rows, int ncells, const uint16_t* iq,
                     const float* iw, float* scores, int64_t ld, void* stream);
@@ -171,7 +204,7 @@ size_t qsa_topk_workspace_bytes(int rows, int L, int top_k);
  * score, equal scores going to the lower index, all visible cells when fewer
  * than top_k: ids[r][0..top_k) ascending, padded with -1.  The order is exact
  * on the fp32 values (radix select on order-preserving 32-bit keys; -0 == +0).
- * Requires vis0 >= 1, vis0 + rows - 1 <= ld, ld % 4 == 0.
+ * Requires 1 <= rows <= QSA_MAX_ROWS, vis0 >= 1, vis0 + rows - 1 <= ld, ld % 4 == 0.
  */
 int qsa_topk(const float* scores, int64_t ld, int rows, int vis0, int top_k, void* ws,
              size_t ws_bytes, int32_t* ids, void* stream);
@@ -183,22 +216,25 @@ int qsa_topk(const float* scores, int64_t ld, int rows, int vis0, int top_k, voi
  * < 0 skipped:
  *   s_c = scale * sum_d q[r][h][d] * k[c][g][d] * ks[c][g][d/32]
  *   m = max_c s_c, l = sum_c exp(s_c - m), o = sum_c exp(s_c - m) * v[c][g][:] * vs[c][g][:/32]
- * nsplit == 1: out[r][h][:] = o / l (0 for an empty list); part unused.
+ * nsplit == 1: out[r][h][:] = o / l (0 for an empty list), times sigmoid(gate[r][h][:])
+ *              when gate (fp32 [rows][24][256]) is not NULL; part unused.
  * nsplit > 1:  part[((r * 24 + h) * nsplit + j) * 258 + {0, 1, 2..257}] = {m, l, o}
- *              (m = -inf, l = 0, o = 0 for an empty piece); out unused.
+ *              (m = -inf, l = 0, o = 0 for an empty piece); out and gate unused.
  * Query and P are rounded to fp16 for the tensor cores; K/V codes are exact;
- * accumulation is fp32.  Requires 1 <= nsplit <= 64, ids < max_cells.
+ * accumulation is fp32.  Requires 1 <= rows <= QSA_MAX_ROWS, 1 <= nsplit <= 64;
+ * ids outside [0, max_cells) count as empty slots.
  */
 int qsa_attn(const qsa_cache* cache, int rows, const float* q, const int32_t* ids, int top_k,
-             int nsplit, float scale, float* part, float* out, void* stream);
+             int nsplit, float scale, const float* gate, float* part, float* out, void* stream);
 
 /*
  * Step 4, log-sum-exp merge (qsa_merge: "opus r20 track A ...", section 2):
  * per row and head, M = max m_j over pieces with l_j > 0, e_j = exp(m_j - M),
- * L = sum_j l_j e_j and o = sum_j o_j e_j, both in j order, out = o / L
- * (0 when every piece is empty).  part as written by qsa_attn.
+ * L = sum_j l_j e_j and o = sum_j o_j e_j, out = o / L (0 when every piece is
+ * empty), times sigmoid(gate[r][h][:]) when gate (fp32 [rows][24][256]) is not
+ * NULL.  part as written by qsa_attn.
  */
-int qsa_merge(const float* part, int rows, int nsplit, float* out, void* stream);
+int qsa_merge(const float* part, int rows, int nsplit, const float* gate, float* out, void* stream);
 
 /*
  * Selection without a caller workspace.  The pages have no counterpart to this
@@ -231,7 +267,7 @@ int qsa_topk_static(const float* scores, int64_t ld, int rows, int vis0, int top
 
 /*
  * Device-side failure report.  Kernels that wait on an mbarrier (the prefill
- * score GEMM) bound every wait to one second; on expiry they stop, drain their
+ * score GEMM) bound every wait to four seconds; on expiry they stop, drain their
  * copies, free their tensor memory and record QSA_ERR_TIMEOUT in a status word
  * of the current device.  This call copies that word into *status (QSA_OK or
  * QSA_ERR_TIMEOUT) and clears it.  Unlike the other calls it synchronises
@@ -246,6 +282,20 @@ int qsa_device_status(int* status, void* stream);
  * usable.
  */
 int qsa_selftest_wait_timeout(void* stream);
+
+/*
+ * Per-kernel timing of this thread's calls (the pages time each dispatch on the GPU:
+ * "opus r20 track A ...", section 4).  qsa_trace_begin records a start event on
+ * `stream`; until qsa_trace_end, every kernel this thread's calls launch is followed by
+ * an event on that stream (so trace calls made on that stream; the events also end the
+ * overlap of consecutive kernels, so the times are those of kernels run back to back).
+ * qsa_trace_end stops tracing, waits for the last event (it synchronises) and returns
+ * the number of launches in *n and, for the first min(*n, cap), the milliseconds from
+ * the previous event in ms[i] and the kernel's name in names[i] (static strings; either
+ * array may be NULL).  capacity: 1 .. 4096 launches; later ones are not timed.
+ */
+int qsa_trace_begin(int capacity, void* stream);
+int qsa_trace_end(int cap, int* n, float* ms, const char** names);
 
 /* Text of the last error on the calling thread ("" when none). */
 const char* qsa_last_error(void);

@@ -57,8 +57,11 @@ def test_workspace_bytes(lib):
     b = lib.qsa_workspace_bytes(0, 1, 65536, 512, 1)
     c = lib.qsa_workspace_bytes(0, 1, 65536, 512, 64)
     assert 0 < a < b < c
-    # scores alone need rows * L * 4 bytes
-    assert lib.qsa_workspace_bytes(1, 1024, 262144, 2048, 0) >= 1024 * 262144 * 4
+    # a decode step holds its rows' scores (rows * L * 4 bytes); a prompt chunk of more than
+    # 8 rows holds candidate lists instead, well under its T x L score matrix
+    assert lib.qsa_workspace_bytes(0, 8, 262144, 2048, 0) >= 8 * 262144 * 4
+    pre = lib.qsa_workspace_bytes(1, 1024, 262144, 2048, 0)
+    assert 0 < pre < 1024 * 262144 * 4 // 2
     assert lib.qsa_topk_workspace_bytes(4, 1000, 100) > 4 * 2048 * 4
 
 
@@ -66,8 +69,10 @@ def test_decode_rejects_bad_arguments(lib):
     from top_sparse_attention_score_b200 import qsa
     cs = _fake_cache(qsa)
     P = ctypes.c_void_p(0x60000)
-    def call(L=1000, n=1, top_k=64, nsplit=0, ws_bytes=1 << 40, q=P, cache=ctypes.byref(cs)):
-        return lib.qsa_decode(cache, L, n, q, P, P, top_k, nsplit, 0.0625, P, ws_bytes, P, None, None)
+    def call(L=1000, n=1, top_k=64, nsplit=0, ws_bytes=1 << 40, q=P, cache=ctypes.byref(cs), append=None,
+             gate=None):
+        return lib.qsa_decode(cache, L, n, append, q, P, P, gate, top_k, nsplit, 0.0625, P, ws_bytes, P, None,
+                              None)
     assert call(n=0) == 1 and "n = 0" in qsa.last_error()
     assert call(n=9) == 1
     assert call(L=1001) == 1                      # beyond max_cells
@@ -81,6 +86,9 @@ def test_decode_rejects_bad_arguments(lib):
     assert call(cache=None) == 1
     bad = qsa.CacheStruct(0x10000, 0, 0x30000, 0x40000, 0x50000, 1000)
     assert call(cache=ctypes.byref(bad)) == 1
+    half = qsa.NewCellsStruct(0x70000, 0, 0x80000)                # append with a NULL array
+    assert call(append=ctypes.byref(half)) == 1 and "append" in qsa.last_error()
+    assert call(gate=ctypes.c_void_p(0x60008)) == 1               # misaligned gate
 
 
 def test_prefill_and_steps_reject_bad_arguments(lib):
@@ -88,9 +96,13 @@ def test_prefill_and_steps_reject_bad_arguments(lib):
     cs = _fake_cache(qsa)
     P = ctypes.c_void_p(0x60000)
     cb = ctypes.byref(cs)
-    assert lib.qsa_prefill_chunk(cb, 990, 20, P, P, P, 64, 0.0625, P, 1 << 40, P, None, None) == 1
-    assert lib.qsa_prefill_chunk(cb, -1, 20, P, P, P, 64, 0.0625, P, 1 << 40, P, None, None) == 1
-    assert lib.qsa_prefill_chunk(cb, 0, 20, P, P, P, 64, 0.0625, P, 10, P, None, None) == 2
+    def prefill(pos0, T, ws_bytes=1 << 40, cache=cb):
+        return lib.qsa_prefill_chunk(cache, pos0, T, None, P, P, P, None, 64, 0.0625, P, ws_bytes, P, None, None)
+    assert prefill(990, 20) == 1
+    assert prefill(-1, 20) == 1
+    assert prefill(0, 20, ws_bytes=10) == 2
+    big = qsa.CacheStruct(0x10000, 0x20000, 0x30000, 0x40000, 0x50000, 1 << 20)
+    assert prefill(0, 65536, cache=ctypes.byref(big)) == 1 and "65535" in qsa.last_error()  # grid limit
     assert lib.qsa_cache_write(cb, 999, 2, P, P, P, None) == 1
     assert lib.qsa_cache_write(cb, 0, 0, P, P, P, None) == 1
     assert lib.qsa_index_score(cb, 1, 100, P, P, P, 99, None) == 1       # ld < ncells
@@ -99,11 +111,13 @@ def test_prefill_and_steps_reject_bad_arguments(lib):
     assert lib.qsa_topk(P, 100, 2, 100, 10, P, 1 << 40, P, None) == 1    # row 1 sees 101 > ld
     assert lib.qsa_topk(P, 100, 1, 0, 10, P, 1 << 40, P, None) == 1      # vis0 < 1
     assert lib.qsa_topk(P, 100, 1, 50, 10, P, 10, P, None) == 2
-    assert lib.qsa_attn(cb, 1, P, P, 64, 0, 0.0625, P, P, None) == 1
-    assert lib.qsa_attn(cb, 1, P, P, 64, 2, 0.0625, None, P, None) == 1  # nsplit > 1 needs part
-    assert lib.qsa_attn(cb, 1, P, P, 64, 1, 0.0625, P, None, None) == 1  # nsplit 1 needs out
-    assert lib.qsa_merge(None, 1, 2, P, None) == 1
-    assert lib.qsa_merge(P, 1, 65, P, None) == 1
+    assert lib.qsa_topk(P, 1 << 20, 65536, 50, 10, P, 1 << 40, P, None) == 1  # rows above 65535
+    assert lib.qsa_attn(cb, 1, P, P, 64, 0, 0.0625, None, P, P, None) == 1
+    assert lib.qsa_attn(cb, 1, P, P, 64, 2, 0.0625, None, None, P, None) == 1  # nsplit > 1 needs part
+    assert lib.qsa_attn(cb, 1, P, P, 64, 1, 0.0625, None, P, None, None) == 1  # nsplit 1 needs out
+    assert lib.qsa_attn(cb, 65536, P, P, 64, 1, 0.0625, None, P, P, None) == 1  # rows above 65535
+    assert lib.qsa_merge(None, 1, 2, None, P, None) == 1
+    assert lib.qsa_merge(P, 1, 65, None, P, None) == 1
 
 
 def test_bench_split_rule_matches_the_library(lib):

@@ -221,6 +221,16 @@ def test_topk_threshold_bin_sizes(gpu):
     _topk_case(gpu, s, V, k)
 
 
+@pytest.mark.parametrize("V,ties", [(65537, False), (200000, True), (262142, False)])
+def test_topk_wide_cluster(gpu, V, ties):
+    # rows of 65537 .. 262144 cells: one 16-CTA cluster per row (32 cells per thread)
+    st = synth.Stream(109 + V, "tk")
+    s = st.normal(3 * (V + 2)).reshape(3, V + 2)
+    if ties:
+        s = np.round(s * 4) / 4
+    _topk_case(gpu, s.astype(np.float32), V, 2048)
+
+
 def test_topk_many_windows(gpu):
     st = synth.Stream(106, "tk")
     V = (1 << 19) * 2 + 777
@@ -519,14 +529,21 @@ def test_decode_nsplit_invariance(gpu):
         assert rel_err(o, outs[0]) <= SPLIT_TOL
 
 
-def _prefill_case(qsa, wl, rows):
+def _prefill_case(qsa, wl, rows, batch=256):
+    """One GPU chunk; the oracle on the given rows, `batch` rows at a time (its float64
+    scores of a batch are held at once)."""
     cache, q, iq, iw = dev_inputs(qsa, wl)
     ids = torch.empty(wl.rows, wl.top_k, dtype=torch.int32, device=DEV)
     out = qsa.prefill_chunk(cache, wl.pos0, q, iq, iw, wl.top_k, wl.scale, ids_out=ids)
     torch.cuda.synchronize()
-    ref_out, ref_ids, ref_sc = oracle.rows(wl, np.array(rows), want_scores=True, threads=THREADS)
-    return check_outputs(qsa, cache, q, out.cpu().numpy(), ids.cpu().numpy()[rows], ref_out, ref_ids,
-                         ref_sc, rows, wl.scale, wl.top_k)
+    out, ids = out.cpu().numpy(), ids.cpu().numpy()
+    exact = 0
+    for b in range(0, len(rows), batch):
+        part = rows[b:b + batch]
+        ref_out, ref_ids, ref_sc = oracle.rows(wl, np.array(part), want_scores=True, threads=THREADS)
+        exact += check_outputs(qsa, cache, q, out, ids[part], ref_out, ref_ids, ref_sc, part, wl.scale,
+                               wl.top_k)
+    return exact
 
 
 def test_prefill_small_all_rows(gpu):
@@ -535,14 +552,52 @@ def test_prefill_small_all_rows(gpu):
     _prefill_case(gpu, wl, list(range(150)))
 
 
-def test_prefill_config3_sampled(gpu):
+def test_prefill_config3_all_rows(gpu):
+    # T = 2048 at 63488 over 65536 cells: every row, so every 128-token GEMM tile and every
+    # row's selection is compared with the oracle (about 1.3e8 cells of float64 scores)
     wl = synth.make_workload(3)
-    _prefill_case(gpu, wl, [0, 1, 777, 1500, 2046, 2047])
+    _prefill_case(gpu, wl, list(range(wl.rows)))
 
 
-def test_prefill_config4_sampled(gpu):
+def test_prefill_config4_all_rows(gpu):
+    # T = 1024 at 261120 over 262144 cells with 10% duplicated keys (ties): every row
     wl = synth.make_workload(4)
-    _prefill_case(gpu, wl, [0, 511, 1022, 1023])
+    _prefill_case(gpu, wl, list(range(wl.rows)))
+
+
+@pytest.mark.parametrize("T,cells,top_k", [(9, 1500, 128), (65, 3000, 512), (200, 9000, 2048)])
+def test_prefill_ragged_chunks(gpu, T, cells, top_k):
+    # chunks just above 8 rows (the GEMV/cluster path ends there), a token block and one
+    # row, cell counts that are not multiples of the 128-cell tiles
+    wl = synth.make_workload(3, cells=cells, rows=T)
+    wl.top_k = top_k
+    _prefill_case(gpu, wl, list(range(T)))
+
+
+def test_prefill_sample_fooled(gpu):
+    # every 16th cell (the cells the threshold pass samples) has a large key and the rest
+    # small ones: the sampled threshold admits fewer than top_k cells, so every row takes
+    # the exact recomputing path
+    wl = synth.make_workload(3, cells=6000, rows=40)
+    wl.top_k = 512
+    key = wl.cache.idx_key.astype(np.float32)
+    key *= 0.05
+    key[::16] *= 400.0
+    wl.cache.idx_key = key.astype(np.float16)
+    _prefill_case(gpu, wl, list(range(40)))
+
+
+def test_prefill_all_keys_equal(gpu):
+    # identical keys: every visible cell ties, the candidate lists overflow and the exact
+    # path keeps the lowest indices
+    wl = synth.make_workload(3, cells=5000, rows=30)
+    wl.top_k = 700
+    wl.cache.idx_key[:] = wl.cache.idx_key[0]
+    qsa = gpu
+    cache, q, iq, iw = dev_inputs(qsa, wl)
+    ids = torch.empty(30, 700, dtype=torch.int32, device=DEV)
+    qsa.prefill_chunk(cache, wl.pos0, q, iq, iw, 700, wl.scale, ids_out=ids)
+    assert np.array_equal(ids.cpu().numpy(), np.tile(np.arange(700, dtype=np.int32), (30, 1)))
 
 
 def test_prefill_row_equals_decode(gpu):
@@ -567,6 +622,157 @@ def test_prefill_row_equals_decode(gpu):
         if np.array_equal(a, b):
             # prefill picks its own split count; see test_decode_nsplit_invariance
             assert rel_err(out_d.cpu().numpy()[0], out_p.cpu().numpy()[t]) <= SPLIT_TOL
+
+
+def test_attn_softmax_golden(gpu):
+    # the hand-worked softmax fixture through the kernels: weights w_c / sum(w) from
+    # logits ln w_c, outputs 30 and 19.2 (times 2^-(d div 32)), one piece and two pieces
+    from tests import pins
+    qsa = gpu
+    cache_h, q, vals, _ = pins.softmax_golden_case()
+    cache = qsa.DeviceCache.from_host(cache_h, DEV)
+    dims = 2.0 ** -(np.arange(256) // 32)
+    want = np.stack([vals["out"][h // 12] * dims for h in range(24)])
+    ids = torch.arange(4, dtype=torch.int32, device=DEV)[None]
+    qd = torch.from_numpy(q[None]).to(DEV)
+    one = qsa.attn(cache, qd, ids, 1, 1 / 16).cpu().numpy()[0]
+    two = qsa.merge(qsa.attn(cache, qd, ids, 2, 1 / 16)).cpu().numpy()[0]
+    assert rel_err(one, want) <= OUT_TOL and rel_err(two, want) <= OUT_TOL
+
+
+def _gate(seed, rows):
+    return torch.from_numpy((synth.Stream(seed, "gate").normal(rows * 24 * 256) * 2).astype(np.float32)
+                            .reshape(rows, 24, 256)).to(DEV)
+
+
+@pytest.mark.parametrize("nsplit", [1, 6])
+def test_attn_and_merge_gate(gpu, nsplit):
+    # out = O * sigmoid(gate): nsplit 1 gates in the attention epilogue, more pieces in the merge
+    qsa = gpu
+    rows, cells, k = 3, 3000, 256
+    wl = synth.make_workload(0, cells=cells)
+    q, _, _ = synth.make_queries(221, rows)
+    ids = _id_lists(222, rows, cells, k, [256, 100, 1])
+    gate = _gate(223, rows)
+    cache = qsa.DeviceCache.from_host(wl.cache, DEV)
+    qd, idd = torch.from_numpy(q).to(DEV), torch.from_numpy(ids).to(DEV)
+    if nsplit == 1:
+        out = qsa.attn(cache, qd, idd, 1, 1 / 16, gate=gate)
+        plain = qsa.attn(cache, qd, idd, 1, 1 / 16)
+    else:
+        part = qsa.attn(cache, qd, idd, nsplit, 1 / 16)
+        out, plain = qsa.merge(part, gate=gate), qsa.merge(part)
+    out, plain, g = out.cpu().numpy(), plain.cpu().numpy(), gate.cpu().numpy()
+    for r in range(rows):
+        ref = oracle.gate_row(oracle.attn_row(wl.cache, q[r], ids[r], 1 / 16), g[r])
+        assert rel_err(out[r], ref) <= OUT_TOL
+        assert np.allclose(out[r], plain[r] / (1 + np.exp(-g[r].astype(np.float64))), rtol=1e-5, atol=1e-30)
+
+
+@pytest.mark.parametrize("kind", ["decode", "decode_dense", "prefill"])
+def test_step_with_append_and_gate(gpu, kind):
+    # one call appends the rows' own cells (quantized exactly as qsa_cache_write does), then
+    # runs the step and gates the output; bit-equal to a separate cache write plus the step.
+    # Decode appends inside its scoring kernel; the short-context path and prefill chunks
+    # run the cache write first.
+    qsa = gpu
+    if kind.startswith("decode"):
+        wl = synth.make_workload(1, n=6, cells=7000 if kind == "decode" else 400)
+        if kind == "decode_dense":
+            wl.top_k = 512
+        pos = wl.L - wl.rows
+    else:
+        wl = synth.make_workload(3, cells=2600, rows=140)
+        wl.top_k = 256
+        pos = wl.pos0
+    rows = wl.rows
+    kn, vn, keyn = synth.make_new_cells(231, rows)
+    gate = _gate(232, rows)
+    cache, q, iq, iw = dev_inputs(qsa, wl)       # the new cells' slots hold other data
+    twin, _, _, _ = dev_inputs(qsa, wl)
+    app = (torch.from_numpy(kn).to(DEV), torch.from_numpy(vn).to(DEV), torch.from_numpy(keyn).to(DEV))
+    ids = torch.empty(rows, wl.top_k, dtype=torch.int32, device=DEV)
+    ids2 = torch.empty_like(ids)
+    if kind.startswith("decode"):
+        out = qsa.decode(cache, wl.L, q, iq, iw, wl.top_k, 0, wl.scale, ids_out=ids, append=app, gate=gate)
+        qsa.cache_write(twin, pos, *app)
+        out2 = qsa.decode(twin, wl.L, q, iq, iw, wl.top_k, 0, wl.scale, ids_out=ids2, gate=gate)
+    else:
+        out = qsa.prefill_chunk(cache, pos, q, iq, iw, wl.top_k, wl.scale, ids_out=ids, append=app, gate=gate)
+        qsa.cache_write(twin, pos, *app)
+        out2 = qsa.prefill_chunk(twin, pos, q, iq, iw, wl.top_k, wl.scale, ids_out=ids2, gate=gate)
+    torch.cuda.synchronize()
+    for a, b in ((cache.k, twin.k), (cache.v, twin.v), (cache.ks, twin.ks), (cache.vs, twin.vs),
+                 (cache.idx_key, twin.idx_key)):
+        assert torch.equal(a, b)
+    assert torch.equal(ids, ids2)
+    assert np.array_equal(out.cpu().numpy().view(np.uint32), out2.cpu().numpy().view(np.uint32))
+    # against the oracle: its own cache write, then the gated step
+    oracle.cache_write(wl.cache, pos, kn, vn, keyn)
+    assert np.array_equal(cache.k.cpu().numpy(), wl.cache.k)
+    sel = list(range(0, rows, max(1, rows // 10)))
+    ref_out, ref_ids, ref_sc = oracle.rows(wl, np.array(sel), want_scores=True, threads=THREADS,
+                                           gate=gate.cpu().numpy())
+    exact = set(check_selection(ids.cpu().numpy()[sel], ref_ids, ref_sc, wl.top_k))
+    out = out.cpu().numpy()
+    g = gate.cpu().numpy()
+    for i, r in enumerate(sel):
+        if i in exact:
+            got = out[r]
+        else:
+            got = qsa.attn(cache, q[r:r + 1].contiguous(), torch.from_numpy(ref_ids[i:i + 1]).to(DEV), 1,
+                           wl.scale, gate=gate[r:r + 1].contiguous()).cpu().numpy()[0]
+        assert rel_err(got, ref_out[i]) <= OUT_TOL, r
+
+
+SENTINEL = 0x7FC0BEEF  # a NaN bit pattern no kernel writes
+
+
+def _guarded(shape, dtype, pad):
+    """A buffer of `shape` with `pad` guard elements before and after it, all set to the
+    sentinel bits; returns (whole buffer, the view handed to the library)."""
+    n = int(np.prod(shape))
+    whole = torch.full((n + 2 * pad,), SENTINEL, dtype=torch.int32, device=DEV)
+    whole = whole.view(dtype) if dtype != torch.int32 else whole
+    return whole, whole[pad:pad + n].view(*shape)
+
+
+def _guards_intact(whole, pad):
+    bits = whole.view(torch.int32).cpu().numpy()
+    return bool(np.all(bits[:pad] == SENTINEL) and np.all(bits[-pad:] == SENTINEL))
+
+
+@pytest.mark.parametrize("kind", ["decode", "prefill"])
+def test_step_writes_stay_inside_outputs(gpu, kind):
+    # out, ids_out and the workspace each sit between guard regions (a whole row of out
+    # on both sides, 64 ids, 4 KB of workspace): the step must write only inside them
+    qsa = gpu
+    if kind == "decode":
+        wl = synth.make_workload(1, n=5, cells=9000)
+        mode, L = qsa.MODE_DECODE, wl.L
+    else:
+        wl = synth.make_workload(3, cells=2600, rows=140)
+        wl.top_k = 256
+        mode, L = qsa.MODE_PREFILL, wl.pos0 + wl.rows
+    cache, q, iq, iw = dev_inputs(qsa, wl)
+    rows = wl.rows
+    pad_out, pad_ids, pad_ws = 24 * 256, 64, 1024
+    out_w, out = _guarded((rows, 24, 256), torch.float32, pad_out)
+    ids_w, ids = _guarded((rows, wl.top_k), torch.int32, pad_ids)
+    nbytes = qsa.workspace_bytes(mode, rows, L, wl.top_k, wl.nsplit if kind == "decode" else 0)
+    ws_w, ws = _guarded(((nbytes + 3) // 4,), torch.int32, pad_ws)
+    ws = ws.view(torch.uint8)
+    if kind == "decode":
+        qsa.decode(cache, wl.L, q, iq, iw, wl.top_k, wl.nsplit, wl.scale, ws=ws, out=out, ids_out=ids)
+    else:
+        qsa.prefill_chunk(cache, wl.pos0, q, iq, iw, wl.top_k, wl.scale, ws=ws, out=out, ids_out=ids)
+    torch.cuda.synchronize()
+    assert _guards_intact(out_w, pad_out) and _guards_intact(ids_w, pad_ids) and _guards_intact(ws_w, pad_ws)
+    # and the result inside is the step's result
+    sel = list(range(0, rows, max(1, rows // 12)))
+    ref_out, ref_ids, ref_sc = oracle.rows(wl, np.array(sel), want_scores=True, threads=THREADS)
+    check_outputs(qsa, cache, q, out.cpu().numpy(), ids.cpu().numpy()[sel], ref_out, ref_ids, ref_sc, sel,
+                  wl.scale, wl.top_k)
 
 
 def test_errors_and_launch_count(gpu):

@@ -1,12 +1,13 @@
 """The selection call that needs no workspace (qsa_topk_static) against the
-workspace version (qsa_topk), through the C ABI.
+workspace version (qsa_topk) and the CPU oracle, through the C ABI.
 
 It serves callers that cannot allocate device memory at the point of the call
 (inside a CUDA graph capture, in serving loops that must avoid allocator calls
 and their implicit synchronisation, or under a memory budget owned by another
 allocator).  Two calls in a row on different scores must each match qsa_topk
-exactly -- the second also shows the shared scratch buffer is cleared between
-calls.  The file is named to be collected last, and passes both alone in a
+exactly, and the oracle's selection on the same fp32 scores (widened exactly to
+float64, so both decide on the same values) -- the second call also shows the
+shared scratch buffer is cleared between calls.  The file is named to be collected last, and passes both alone in a
 fresh process (where its first call looks up the buffer) and after the others.
 """
 import ctypes
@@ -15,6 +16,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
 
 pytestmark = pytest.mark.gpu
@@ -48,6 +50,10 @@ def test_static_topk_matches_workspace_topk(gpu):
         want = qsa.topk(scores, vis0, top_k)
         torch.cuda.synchronize()
         assert torch.equal(got, want)
+        host, ids = scores.cpu().numpy(), got.cpu().numpy()
+        for r in range(host.shape[0]):
+            ref = oracle.topk(host[r, :vis0 + r].astype(np.float64), top_k)
+            assert np.array_equal(ids[r], ref), r
 
 
 def test_static_topk_rejects_oversize(gpu):

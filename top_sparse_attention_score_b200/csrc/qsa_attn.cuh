@@ -67,6 +67,7 @@ struct AttnArgs {
   float scale_log2;   // softmax scale * log2(e)
   float* part;        // [rows][24][nsplit][258] when nsplit > 1
   float* out;         // [rows][24][256] when nsplit == 1
+  const float* gate;  // [rows][24][256] or NULL: out *= sigmoid(gate) when nsplit == 1
   int dense_vis0;     // ids == NULL: cells row 0 sees (row r sees dense_vis0 + r <= top_k)
   int* ids_fill;      // ids == NULL: optional [rows][top_k] copy of the implicit lists
 };
@@ -79,17 +80,73 @@ __device__ __forceinline__ int attn_cell(const int* rid, int dv, int p, int end)
   else return __ldg(rid + p);
 }
 
-template <int NT, bool kAll>
-__device__ __forceinline__ void attn_issue(AttnStage& st, const AttnArgs& a, const int* rid, int dv, int pos0,
-                                           int end, int kvh) {
-  const int tid = threadIdx.x;
+// ---- pieces shared by attn_kernel and the fused decode kernel
+
+// Online-softmax state of one W-warp group for one (row, KV head): the reference
+// maximum (log2 units) of P, finite from the start so a block with no valid cell gives
+// exp2(-inf - m_run) = 0 without a guard; the true maximum; the weight sum; and this
+// warp's O accumulators (rows g and g + 8 of the 16-row tiles).
+template <int W>
+struct AttnState {
+  static constexpr int GW = kNG / W;  // scale groups (32 dims each) per warp
+  float m_run[2], m_top[2], l_run[2];
+  float o[GW][4][4];
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      m_run[r] = kAttnNoMax;
+      m_top[r] = -INFINITY;
+      l_run[r] = 0.f;
+    }
+#pragma unroll
+    for (int gi = 0; gi < GW; ++gi)
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) o[gi][i][c] = 0.f;
+  }
+};
+
+// Q fragments for warp `warp` of a W-warp group, its kNG / W scale groups of dims, prescaled
+// by sl = scale * log2(e).  q0 points at the KV head's first query head of the row.
+// Within group qg, thread t covers dims 32qg + 8t + 4s + {0..3} in sub-step s:
+// k-index 2t,2t+1 <-> +0,+1 and 2t+8,2t+9 <-> +2,+3 (the same map as the K loads).
+template <int W>
+__device__ __forceinline__ void attn_load_q(uint32_t (&aq)[kNG / W][2][4], const float* q0, float sl, int warp) {
+  constexpr int GW = kNG / W;
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const float* qg0 = q0 + g * kD;
+  const float* q8 = qg0 + 8 * kD;
+  const bool has8 = g + 8 < kQPerKV;
+#pragma unroll
+  for (int gi = 0; gi < GW; ++gi)
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      const int d0 = 32 * (GW * warp + gi) + 8 * t + 4 * s;
+      const float4 x = __ldg(reinterpret_cast<const float4*>(qg0 + d0));
+      aq[gi][s][0] = pack_half2(x.x * sl, x.y * sl);
+      aq[gi][s][2] = pack_half2(x.z * sl, x.w * sl);
+      if (has8) {
+        const float4 y = __ldg(reinterpret_cast<const float4*>(q8 + d0));
+        aq[gi][s][1] = pack_half2(y.x * sl, y.y * sl);
+        aq[gi][s][3] = pack_half2(y.z * sl, y.w * sl);
+      } else {
+        aq[gi][s][1] = 0u;
+        aq[gi][s][3] = 0u;
+      }
+    }
+}
+
+// Gather one block of 32 cells into `st` with NT threads (tid = 0 .. NT - 1): slot i holds
+// cell cell_of(i), an empty slot for one < 0 or >= max_cells.
+template <int NT, class CellOf>
+__device__ __forceinline__ void attn_gather(AttnStage& st, const AttnArgs& a, int kvh, int tid, CellOf cell_of) {
   // K and V rows: 32 cells x 16 chunks of 16 bytes each, 512 / NT + 512 / NT per thread.
 #pragma unroll
   for (int u = 0; u < 512 / NT; ++u) {
     const int chunk = tid + NT * u;
     const int i = chunk >> 4, part = chunk & 15;
-    const int p = pos0 + i;
-    int cell = attn_cell<kAll>(rid, dv, p, end);
+    int cell = cell_of(i);
     const bool ok = cell >= 0 && cell < a.max_cells;
     if (!ok) cell = 0;
     const size_t row = (static_cast<size_t>(cell) * kHKV + kvh) * kD + part * 16;
@@ -98,8 +155,7 @@ __device__ __forceinline__ void attn_issue(AttnStage& st, const AttnArgs& a, con
   }
   if (tid < 2 * kAttnCells) {  // scales: 64 rows of 16 bytes
     const int i = tid & 31;
-    const int p = pos0 + i;
-    int cell = attn_cell<kAll>(rid, dv, p, end);
+    int cell = cell_of(i);
     const bool ok = cell >= 0 && cell < a.max_cells;
     if (tid < kAttnCells) st.valid[i] = ok;
     if (!ok) cell = 0;
@@ -109,11 +165,152 @@ __device__ __forceinline__ void attn_issue(AttnStage& st, const AttnArgs& a, con
   }
 }
 
+// One gathered block through the online softmax, for warp `warp` of a W-warp group:
+// partial QK^T over the warp's dims, the group's partial scores summed through `red`
+// (every warp in the same order, so all agree bit for bit), masking, the running
+// maximum, the weights and P.V into the warp's O.  `sync` is the group's barrier.
+template <int W, class Sync>
+__device__ __forceinline__ void attn_block(const AttnStage& st, float4 (*red)[4][32],
+                                           const uint32_t (&aq)[kNG / W][2][4], AttnState<W>& S, int warp,
+                                           Sync sync) {
+  constexpr int GW = kNG / W;
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const uint32_t valid = __ballot_sync(0xffffffffu, st.valid[lane] != 0);  // bit c: slot c holds a cell
+
+  // ---- partial scores over this warp's dims
+  float s[4][4];
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) s[nt][c] = 0.f;
+    const int8_t* krow = st.k + (8 * nt + g) * kAttnKStride;
+#pragma unroll
+    for (int gi = 0; gi < GW; ++gi) {
+      const int qg = GW * warp + gi;
+      const uint2 kw = *reinterpret_cast<const uint2*>(krow + 32 * qg + 8 * t);
+      const uint32_t x0 = kw.x ^ 0x80808080u, x1 = kw.y ^ 0x80808080u;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      mma_f16_16816(acc, aq[gi][0], i8x2_to_h2(x0, 0x4140u), i8x2_to_h2(x0, 0x4342u));
+      mma_f16_16816(acc, aq[gi][1], i8x2_to_h2(x1, 0x4140u), i8x2_to_h2(x1, 0x4342u));
+      const float2 sc = make_float2(__half2float(st.ks[(8 * nt + 2 * t) * kNG + qg]),
+                                    __half2float(st.ks[(8 * nt + 2 * t + 1) * kNG + qg]));
+      s[nt][0] = fmaf(sc.x, acc[0], s[nt][0]);
+      s[nt][1] = fmaf(sc.y, acc[1], s[nt][1]);
+      s[nt][2] = fmaf(sc.x, acc[2], s[nt][2]);
+      s[nt][3] = fmaf(sc.y, acc[3], s[nt][3]);
+    }
+    red[warp][nt][lane] = make_float4(s[nt][0], s[nt][1], s[nt][2], s[nt][3]);
+  }
+  sync();
+  // ---- full scores (same summation order in every warp), masked
+  float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt) {
+    float4 r;
+    if constexpr (W == 2) {  // own partial + the other warp's (a + b == b + a: both warps agree)
+      const float4 y = red[warp ^ 1][nt][lane];
+      r = make_float4(s[nt][0] + y.x, s[nt][1] + y.y, s[nt][2] + y.z, s[nt][3] + y.w);
+    } else {
+      r = red[0][nt][lane];
+#pragma unroll
+      for (int w = 1; w < W; ++w) {
+        const float4 y = red[w][nt][lane];
+        r.x += y.x;
+        r.y += y.y;
+        r.z += y.z;
+        r.w += y.w;
+      }
+    }
+    const bool v0 = (valid >> (8 * nt + 2 * t)) & 1u, v1 = (valid >> (8 * nt + 2 * t + 1)) & 1u;
+    s[nt][0] = v0 ? r.x : -INFINITY;
+    s[nt][1] = v1 ? r.y : -INFINITY;
+    s[nt][2] = v0 ? r.z : -INFINITY;
+    s[nt][3] = v1 ? r.w : -INFINITY;
+    mx[0] = fmaxf(mx[0], fmaxf(s[nt][0], s[nt][1]));
+    mx[1] = fmaxf(mx[1], fmaxf(s[nt][2], s[nt][3]));
+  }
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+    mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+  }
+  // The reference maximum m_run moves only when a block exceeds it by more
+  // than 2^8 (P <= 256 in fp16), so most blocks skip the rescale of O; the
+  // true maximum m_top is kept for the split partials.
+#pragma unroll
+  for (int r = 0; r < 2; ++r) S.m_top[r] = fmaxf(S.m_top[r], mx[r]);
+  if (__any_sync(0xffffffffu, mx[0] > S.m_run[0] + kAttnShift || mx[1] > S.m_run[1] + kAttnShift)) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const float mnew = fmaxf(S.m_run[r], mx[r]);
+      const float alpha = exp2f(S.m_run[r] - mnew);
+      S.l_run[r] *= alpha;
+      S.m_run[r] = mnew;
+#pragma unroll
+      for (int gi = 0; gi < GW; ++gi)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          S.o[gi][i][2 * r] *= alpha;
+          S.o[gi][i][2 * r + 1] *= alpha;
+        }
+    }
+  }
+  float rs[2] = {0.f, 0.f};
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int r = c >> 1;
+      const float p = exp2f(s[nt][c] - S.m_run[r]);
+      s[nt][c] = p;
+      rs[r] += p;
+    }
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    rs[r] += __shfl_xor_sync(0xffffffffu, rs[r], 1);
+    rs[r] += __shfl_xor_sync(0xffffffffu, rs[r], 2);
+    S.l_run[r] += rs[r];
+  }
+
+  // ---- P.V for this warp's dims; P's k-index j <-> cell 16*s2 + j
+#pragma unroll
+  for (int s2 = 0; s2 < 2; ++s2) {
+    uint32_t pa[4];
+    pa[0] = pack_half2(s[2 * s2][0], s[2 * s2][1]);
+    pa[1] = pack_half2(s[2 * s2][2], s[2 * s2][3]);
+    pa[2] = pack_half2(s[2 * s2 + 1][0], s[2 * s2 + 1][1]);
+    pa[3] = pack_half2(s[2 * s2 + 1][2], s[2 * s2 + 1][3]);
+    const int cA = 16 * s2 + 2 * t;  // cells of k-index 2t, 2t+1, 2t+8, 2t+9
+#pragma unroll
+    for (int gi = 0; gi < GW; ++gi) {
+      const int qg = GW * warp + gi;
+      // column g of n-tile i is dim 32qg + 4g + i
+      const int8_t* vb = st.v + 32 * qg + 4 * g;
+      const uint32_t wA = *reinterpret_cast<const uint32_t*>(vb + cA * kAttnVStride) ^ 0x80808080u;
+      const uint32_t wB = *reinterpret_cast<const uint32_t*>(vb + (cA + 1) * kAttnVStride) ^ 0x80808080u;
+      const uint32_t wC = *reinterpret_cast<const uint32_t*>(vb + (cA + 8) * kAttnVStride) ^ 0x80808080u;
+      const uint32_t wD = *reinterpret_cast<const uint32_t*>(vb + (cA + 9) * kAttnVStride) ^ 0x80808080u;
+      const __half2 sAB = __halves2half2(st.vs[cA * kNG + qg], st.vs[(cA + 1) * kNG + qg]);
+      const __half2 sCD = __halves2half2(st.vs[(cA + 8) * kNG + qg], st.vs[(cA + 9) * kNG + qg]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint32_t b0 = i8_pair_to_h2(wA, wB, i);
+        uint32_t b1 = i8_pair_to_h2(wC, wD, i);
+        const __half2 h0 = __hmul2(*reinterpret_cast<const __half2*>(&b0), sAB);
+        const __half2 h1 = __hmul2(*reinterpret_cast<const __half2*>(&b1), sCD);
+        mma_f16_16816(S.o[gi][i], pa, *reinterpret_cast<const uint32_t*>(&h0),
+                      *reinterpret_cast<const uint32_t*>(&h1));
+      }
+    }
+  }
+}
+
 // grid: (nsplit, 2, rows); block: 32 * W threads; dynamic smem: sizeof(AttnSmem<W>).
 // kAll: a.ids is NULL and every row's list is all its visible cells.
 template <int W, bool kAll>
 __global__ void __launch_bounds__(32 * W) attn_kernel(AttnArgs a) {
   constexpr int NT = 32 * W;
+  constexpr int GW = kNG / W;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   AttnSmem<W>& sm = *reinterpret_cast<AttnSmem<W>*>(smem_raw);
   const int split = blockIdx.x, kvh = blockIdx.y, row = blockIdx.z;
@@ -126,34 +323,8 @@ __global__ void __launch_bounds__(32 * W) attn_kernel(AttnArgs a) {
   const int nblk = (end - beg + kAttnCells - 1) / kAttnCells;
   griddep_launch();
 
-  // Q fragments for this warp's four scale groups (dims [128w, 128w+128)), prescaled.
-  // Within group qg, thread t covers dims 32qg + 8t + 4s + {0..3} in sub-step s:
-  // k-index 2t,2t+1 <-> +0,+1 and 2t+8,2t+9 <-> +2,+3 (the same map as the K loads).
-  constexpr int GW = kNG / W;  // scale groups (32 dims each) per warp
   uint32_t aq[GW][2][4];
-  {
-    const float* q0 = a.q + (static_cast<size_t>(row) * kHQ + kvh * kQPerKV + g) * kD;
-    const float* q8 = q0 + 8 * kD;
-    const bool has8 = g + 8 < kQPerKV;
-#pragma unroll
-    for (int gi = 0; gi < GW; ++gi)
-#pragma unroll
-      for (int s = 0; s < 2; ++s) {
-        const int d0 = 32 * (GW * warp + gi) + 8 * t + 4 * s;
-        const float4 x = __ldg(reinterpret_cast<const float4*>(q0 + d0));
-        const float sl = a.scale_log2;
-        aq[gi][s][0] = pack_half2(x.x * sl, x.y * sl);
-        aq[gi][s][2] = pack_half2(x.z * sl, x.w * sl);
-        if (has8) {
-          const float4 y = __ldg(reinterpret_cast<const float4*>(q8 + d0));
-          aq[gi][s][1] = pack_half2(y.x * sl, y.y * sl);
-          aq[gi][s][3] = pack_half2(y.z * sl, y.w * sl);
-        } else {
-          aq[gi][s][1] = 0u;
-          aq[gi][s][3] = 0u;
-        }
-      }
-  }
+  attn_load_q<W>(aq, a.q + (static_cast<size_t>(row) * kHQ + kvh * kQPerKV) * kD, a.scale_log2, warp);
 
   // The ids come from the selection kernel: wait for it before the first gather.
   griddep_wait();
@@ -162,161 +333,27 @@ __global__ void __launch_bounds__(32 * W) attn_kernel(AttnArgs a) {
       for (int p = beg + static_cast<int>(threadIdx.x); p < end; p += NT)
         a.ids_fill[static_cast<size_t>(row) * a.top_k + p] = p < dv ? p : -1;
   }
+  auto gather = [&](int blk) {
+    const int p0 = beg + blk * kAttnCells;
+    attn_gather<NT>(sm.st[blk % kAttnStages], a, kvh, static_cast<int>(threadIdx.x),
+                    [&](int i) { return attn_cell<kAll>(rid, dv, p0 + i, end); });
+  };
 #pragma unroll
   for (int st = 0; st < kAttnStages - 1; ++st) {
-    if (st < nblk) attn_issue<NT, kAll>(sm.st[st], a, rid, dv, beg + st * kAttnCells, end, kvh);
+    if (st < nblk) gather(st);
     cp_async_commit();
   }
 
-  // reference maximum (log2 units) of P: finite from the start, so a block with
-  // no valid cell gives exp2(-inf - m_run) = 0 without a guard
-  float m_run[2] = {kAttnNoMax, kAttnNoMax};
-  float m_top[2] = {-INFINITY, -INFINITY};  // true maximum
-  float l_run[2] = {0.f, 0.f};
-  float o[GW][4][4];
-#pragma unroll
-  for (int gi = 0; gi < GW; ++gi)
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) o[gi][i][c] = 0.f;
-
+  AttnState<W> S;
+  S.init();
   for (int b = 0; b < nblk; ++b) {
     // refill the stage block b - 1 used (every warp finished it at the last barrier)
     const int nb = b + kAttnStages - 1;
-    if (nb < nblk) attn_issue<NT, kAll>(sm.st[nb % kAttnStages], a, rid, dv, beg + nb * kAttnCells, end, kvh);
+    if (nb < nblk) gather(nb);
     cp_async_commit();
     cp_async_wait<kAttnStages - 1>();
     __syncthreads();
-    const AttnStage& st = sm.st[b % kAttnStages];
-    const uint32_t valid = __ballot_sync(0xffffffffu, st.valid[lane] != 0);  // bit c: slot c holds a cell
-
-    // ---- partial scores over this warp's 64 dims
-    float s[4][4];
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-#pragma unroll
-      for (int c = 0; c < 4; ++c) s[nt][c] = 0.f;
-      const int8_t* krow = st.k + (8 * nt + g) * kAttnKStride;
-#pragma unroll
-      for (int gi = 0; gi < GW; ++gi) {
-        const int qg = GW * warp + gi;
-        const uint2 kw = *reinterpret_cast<const uint2*>(krow + 32 * qg + 8 * t);
-        const uint32_t x0 = kw.x ^ 0x80808080u, x1 = kw.y ^ 0x80808080u;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        mma_f16_16816(acc, aq[gi][0], i8x2_to_h2(x0, 0x4140u), i8x2_to_h2(x0, 0x4342u));
-        mma_f16_16816(acc, aq[gi][1], i8x2_to_h2(x1, 0x4140u), i8x2_to_h2(x1, 0x4342u));
-        const float2 sc = make_float2(__half2float(st.ks[(8 * nt + 2 * t) * kNG + qg]),
-                                      __half2float(st.ks[(8 * nt + 2 * t + 1) * kNG + qg]));
-        s[nt][0] = fmaf(sc.x, acc[0], s[nt][0]);
-        s[nt][1] = fmaf(sc.y, acc[1], s[nt][1]);
-        s[nt][2] = fmaf(sc.x, acc[2], s[nt][2]);
-        s[nt][3] = fmaf(sc.y, acc[3], s[nt][3]);
-      }
-      sm.red[warp][nt][lane] = make_float4(s[nt][0], s[nt][1], s[nt][2], s[nt][3]);
-    }
-    __syncthreads();
-    // ---- full scores (same summation order in every warp), masked
-    float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-      float4 r;
-      if constexpr (W == 2) {  // own partial + the other warp's (a + b == b + a: both warps agree)
-        const float4 y = sm.red[warp ^ 1][nt][lane];
-        r = make_float4(s[nt][0] + y.x, s[nt][1] + y.y, s[nt][2] + y.z, s[nt][3] + y.w);
-      } else {
-        r = sm.red[0][nt][lane];
-#pragma unroll
-        for (int w = 1; w < W; ++w) {
-          const float4 y = sm.red[w][nt][lane];
-          r.x += y.x;
-          r.y += y.y;
-          r.z += y.z;
-          r.w += y.w;
-        }
-      }
-      const bool v0 = (valid >> (8 * nt + 2 * t)) & 1u, v1 = (valid >> (8 * nt + 2 * t + 1)) & 1u;
-      s[nt][0] = v0 ? r.x : -INFINITY;
-      s[nt][1] = v1 ? r.y : -INFINITY;
-      s[nt][2] = v0 ? r.z : -INFINITY;
-      s[nt][3] = v1 ? r.w : -INFINITY;
-      mx[0] = fmaxf(mx[0], fmaxf(s[nt][0], s[nt][1]));
-      mx[1] = fmaxf(mx[1], fmaxf(s[nt][2], s[nt][3]));
-    }
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
-      mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
-    }
-    // The reference maximum m_run moves only when a block exceeds it by more
-    // than 2^8 (P <= 256 in fp16), so most blocks skip the rescale of O; the
-    // true maximum m_top is kept for the split partials.
-#pragma unroll
-    for (int r = 0; r < 2; ++r) m_top[r] = fmaxf(m_top[r], mx[r]);
-    if (__any_sync(0xffffffffu, mx[0] > m_run[0] + kAttnShift || mx[1] > m_run[1] + kAttnShift)) {
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const float mnew = fmaxf(m_run[r], mx[r]);
-        const float alpha = exp2f(m_run[r] - mnew);
-        l_run[r] *= alpha;
-        m_run[r] = mnew;
-#pragma unroll
-        for (int gi = 0; gi < GW; ++gi)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            o[gi][i][2 * r] *= alpha;
-            o[gi][i][2 * r + 1] *= alpha;
-          }
-      }
-    }
-    float rs[2] = {0.f, 0.f};
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int r = c >> 1;
-        const float p = exp2f(s[nt][c] - m_run[r]);
-        s[nt][c] = p;
-        rs[r] += p;
-      }
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      rs[r] += __shfl_xor_sync(0xffffffffu, rs[r], 1);
-      rs[r] += __shfl_xor_sync(0xffffffffu, rs[r], 2);
-      l_run[r] += rs[r];
-    }
-
-    // ---- P.V for this warp's 64 dims; P's k-index j <-> cell 16*s2 + j
-#pragma unroll
-    for (int s2 = 0; s2 < 2; ++s2) {
-      uint32_t pa[4];
-      pa[0] = pack_half2(s[2 * s2][0], s[2 * s2][1]);
-      pa[1] = pack_half2(s[2 * s2][2], s[2 * s2][3]);
-      pa[2] = pack_half2(s[2 * s2 + 1][0], s[2 * s2 + 1][1]);
-      pa[3] = pack_half2(s[2 * s2 + 1][2], s[2 * s2 + 1][3]);
-      const int cA = 16 * s2 + 2 * t;  // cells of k-index 2t, 2t+1, 2t+8, 2t+9
-#pragma unroll
-      for (int gi = 0; gi < GW; ++gi) {
-        const int qg = GW * warp + gi;
-        // column g of n-tile i is dim 32qg + 4g + i
-        const int8_t* vb = st.v + 32 * qg + 4 * g;
-        const uint32_t wA = *reinterpret_cast<const uint32_t*>(vb + cA * kAttnVStride) ^ 0x80808080u;
-        const uint32_t wB = *reinterpret_cast<const uint32_t*>(vb + (cA + 1) * kAttnVStride) ^ 0x80808080u;
-        const uint32_t wC = *reinterpret_cast<const uint32_t*>(vb + (cA + 8) * kAttnVStride) ^ 0x80808080u;
-        const uint32_t wD = *reinterpret_cast<const uint32_t*>(vb + (cA + 9) * kAttnVStride) ^ 0x80808080u;
-        const __half2 sAB = __halves2half2(st.vs[cA * kNG + qg], st.vs[(cA + 1) * kNG + qg]);
-        const __half2 sCD = __halves2half2(st.vs[(cA + 8) * kNG + qg], st.vs[(cA + 9) * kNG + qg]);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          uint32_t b0 = i8_pair_to_h2(wA, wB, i);
-          uint32_t b1 = i8_pair_to_h2(wC, wD, i);
-          const __half2 h0 = __hmul2(*reinterpret_cast<const __half2*>(&b0), sAB);
-          const __half2 h1 = __hmul2(*reinterpret_cast<const __half2*>(&b1), sCD);
-          mma_f16_16816(o[gi][i], pa, *reinterpret_cast<const uint32_t*>(&h0),
-                        *reinterpret_cast<const uint32_t*>(&h1));
-        }
-      }
-    }
+    attn_block<W>(sm.st[b % kAttnStages], sm.red, aq, S, warp, [] { __syncthreads(); });
     __syncthreads();
   }
   cp_async_wait<0>();
@@ -333,18 +370,24 @@ __global__ void __launch_bounds__(32 * W) attn_kernel(AttnArgs a) {
 #pragma unroll
     for (int gi = 0; gi < GW; ++gi) {
       const int dbase = 32 * (GW * warp + gi) + 8 * t;
-      float4 lo = make_float4(o[gi][0][2 * r], o[gi][1][2 * r], o[gi][2][2 * r], o[gi][3][2 * r]);
-      float4 hi = make_float4(o[gi][0][2 * r + 1], o[gi][1][2 * r + 1], o[gi][2][2 * r + 1],
-                              o[gi][3][2 * r + 1]);
+      float4 lo = make_float4(S.o[gi][0][2 * r], S.o[gi][1][2 * r], S.o[gi][2][2 * r], S.o[gi][3][2 * r]);
+      float4 hi = make_float4(S.o[gi][0][2 * r + 1], S.o[gi][1][2 * r + 1], S.o[gi][2][2 * r + 1],
+                              S.o[gi][3][2 * r + 1]);
       if (a.nsplit == 1) {
-        const float inv = l_run[r] > 0.f ? 1.f / l_run[r] : 0.f;
+        const float inv = S.l_run[r] > 0.f ? 1.f / S.l_run[r] : 0.f;
         lo.x *= inv; lo.y *= inv; lo.z *= inv; lo.w *= inv;
         hi.x *= inv; hi.y *= inv; hi.z *= inv; hi.w *= inv;
+        if (a.gate) {
+          const float4 ga = __ldg(reinterpret_cast<const float4*>(a.gate + rh * kD + dbase));
+          const float4 gb = __ldg(reinterpret_cast<const float4*>(a.gate + rh * kD + dbase + 4));
+          lo.x *= gate_factor(ga.x); lo.y *= gate_factor(ga.y); lo.z *= gate_factor(ga.z); lo.w *= gate_factor(ga.w);
+          hi.x *= gate_factor(gb.x); hi.y *= gate_factor(gb.y); hi.z *= gate_factor(gb.z); hi.w *= gate_factor(gb.w);
+        }
         float* dst = a.out + rh * kD + dbase;
         *reinterpret_cast<float4*>(dst) = lo;
         *reinterpret_cast<float4*>(dst + 4) = hi;
       } else {  // partials relative to the true maximum
-        const float corr = (m_top[r] == -INFINITY) ? 0.f : exp2f(m_run[r] - m_top[r]);
+        const float corr = (S.m_top[r] == -INFINITY) ? 0.f : exp2f(S.m_run[r] - S.m_top[r]);
         lo.x *= corr; lo.y *= corr; lo.z *= corr; lo.w *= corr;
         hi.x *= corr; hi.y *= corr; hi.z *= corr; hi.w *= corr;
         float* dst = a.part + (rh * a.nsplit + split) * kPart;
@@ -353,8 +396,8 @@ __global__ void __launch_bounds__(32 * W) attn_kernel(AttnArgs a) {
         *reinterpret_cast<float2*>(dst + 2 + dbase + 4) = make_float2(hi.x, hi.y);
         *reinterpret_cast<float2*>(dst + 2 + dbase + 6) = make_float2(hi.z, hi.w);
         if (warp == 0 && t == 0) {
-          dst[0] = m_top[r] == -INFINITY ? -INFINITY : m_top[r] * kLn2;
-          dst[1] = l_run[r] * corr;
+          dst[0] = S.m_top[r] == -INFINITY ? -INFINITY : S.m_top[r] * kLn2;
+          dst[1] = S.l_run[r] * corr;
         }
       }
     }

@@ -52,6 +52,10 @@ __device__ __forceinline__ uint32_t i8_pair_to_h2(uint32_t xa, uint32_t xb, int 
   return i8x2_to_h2(t, 0x4140u);
 }
 
+// The output gate ("attention + gate"): the attention output is multiplied
+// elementwise by sigmoid(g) = 1 / (1 + exp(-g)).
+__device__ __forceinline__ float gate_factor(float g) { return 1.f / (1.f + expf(-g)); }
+
 // Order-preserving 32-bit key of an fp32 score: larger value -> larger key,
 // -0 mapped to +0 so the two compare equal.
 __device__ __forceinline__ uint32_t score_key(float f) {
@@ -60,15 +64,17 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-// Coarse bin of a score: the top 11 bits of the order-preserving key of its
-// fp16 rounding.  fp32 -> fp16 round-to-nearest never reverses an order, so a
-// higher bin always holds strictly larger scores.
-__device__ __forceinline__ uint32_t score_bin(float f) {
+// 16-bit order-preserving key of a score's fp16 rounding (-0 mapped to +0).
+// fp32 -> fp16 round-to-nearest never reverses an order, so a bin made of this
+// key's top bits always holds strictly larger scores than every lower bin.
+__device__ __forceinline__ uint32_t score_key16(float f) {
   uint32_t b = __half_as_ushort(__float2half_rn(f));
   if ((b & 0x7fffu) == 0u) b = 0u;
-  const uint32_t k = (b & 0x8000u) ? (~b & 0xffffu) : (b | 0x8000u);
-  return k >> 5;
+  return (b & 0x8000u) ? (~b & 0xffffu) : (b | 0x8000u);
 }
+
+// Coarse bin of a score: the top 11 bits of score_key16 (2048 bins).
+__device__ __forceinline__ uint32_t score_bin(float f) { return score_key16(f) >> 5; }
 
 // Exclusive prefix sum over the block (NT threads, NT % 32 == 0, NT <= 1024).
 // `scratch` is 33 words of shared memory; `total` receives the block sum.

@@ -1,10 +1,18 @@
-// qsa_merge.cuh -- log-sum-exp merge of split partials.
+// qsa_merge.cuh -- log-sum-exp merge of split partials, with the optional output gate.
 //
-// qsa_merge of "opus r20 track A: MTP map mlock + qsa_attn / qsa_merge decode tweaks",
-// section 2: the chunk maxima are loaded once, M = max_k m_k, e_k = exp(m_k - M) is
-// computed once per piece, L = sum_k l_k e_k is summed with fma in piece order by one
-// thread, every thread accumulates o = sum_k o_k e_k with fma in piece order for its
-// dim, and the result is o / L.  Pieces with l = 0 (no cells) are skipped.
+// The merge of qsa_merge ("opus r20 track A: MTP map mlock + qsa_attn / qsa_merge decode
+// tweaks", section 2) rests on the log-sum-exp identity: piece j reports its maximum
+// logit m_j, its weight sum l_j and its unnormalised output o_j, all relative to m_j;
+// rescaled to the common maximum M = max_j m_j by e_j = exp(m_j - M), the pieces add
+// up to L = sum_j l_j e_j and O = sum_j o_j e_j, and the attention output is O / L.
+// Pieces without cells (l_j = 0) contribute nothing and do not set M.
+//
+// The optional gate multiplies the result by sigmoid(gate) elementwise ("attention +
+// gate" in the same page's section 3).
+//
+// One CTA per (row, head), one thread per output dim.  Warp 0 reduces the piece
+// statistics (two pieces per lane, warp-shuffle maximum and sum); every thread has
+// its dim's 64 possible o_j loads in flight before the weights are known.
 #pragma once
 
 #include "qsa_common.cuh"
@@ -13,38 +21,50 @@ namespace qsa {
 
 // grid: rows * 24 (one CTA per row and head); block: 256 threads (one per dim).
 __global__ void __launch_bounds__(256) merge_kernel(const float* __restrict__ part, int nsplit,
+                                                    const float* __restrict__ gate,
                                                     float* __restrict__ out) {
-  __shared__ float sm[64], sl[64], se[64];
-  __shared__ float sL;
+  __shared__ float s_e[64];  // e_j, 0 for empty pieces
+  __shared__ float s_inv;    // 1 / L, 0 when every piece is empty
   const int tid = threadIdx.x;
-  const float* base = part + static_cast<size_t>(blockIdx.x) * nsplit * kPart;
+  const size_t rh = blockIdx.x;
+  const float* base = part + rh * nsplit * kPart;
   griddep_launch();
   griddep_wait();  // the partials come from the attention kernel
-  // every o_j of this dim in flight at once (nsplit <= 64)
   float ov[64];
 #pragma unroll
   for (int j = 0; j < 64; ++j) ov[j] = j < nsplit ? __ldcg(base + j * kPart + 2 + tid) : 0.f;
-  if (tid < nsplit) {
-    sm[tid] = __ldcg(base + tid * kPart + 0);
-    sl[tid] = __ldcg(base + tid * kPart + 1);
+  const float g = gate ? __ldg(gate + rh * kD + tid) : 0.f;
+  if (tid < 32) {
+    float m[2], l[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int j = tid + 32 * u;
+      m[u] = j < nsplit ? __ldcg(base + j * kPart) : -INFINITY;
+      l[u] = j < nsplit ? __ldcg(base + j * kPart + 1) : 0.f;
+    }
+    float M = fmaxf(l[0] > 0.f ? m[0] : -INFINITY, l[1] > 0.f ? m[1] : -INFINITY);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float e[2], L = 0.f;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      e[u] = l[u] > 0.f ? expf(m[u] - M) : 0.f;
+      L = fmaf(l[u], e[u], L);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    s_e[tid] = e[0];
+    s_e[tid + 32] = e[1];
+    if (tid == 0) s_inv = L > 0.f ? 1.f / L : 0.f;
   }
   __syncthreads();
-  float M = -INFINITY;
-  for (int j = 0; j < nsplit; ++j)
-    if (sl[j] > 0.f) M = fmaxf(M, sm[j]);
-  if (tid < nsplit) se[tid] = sl[tid] > 0.f ? expf(sm[tid] - M) : 0.f;
-  __syncthreads();
-  if (tid == 0) {
-    float L = 0.f;
-    for (int j = 0; j < nsplit; ++j) L = fmaf(sl[j], se[j], L);
-    sL = L;
-  }
   float o = 0.f;
 #pragma unroll
   for (int j = 0; j < 64; ++j)
-    if (j < nsplit) o = fmaf(ov[j], se[j], o);
-  __syncthreads();
-  out[static_cast<size_t>(blockIdx.x) * kD + tid] = sL > 0.f ? o / sL : 0.f;
+    if (j < nsplit) o = fmaf(ov[j], s_e[j], o);
+  float r = o * s_inv;
+  if (gate) r *= gate_factor(g);
+  out[rh * kD + tid] = r;
 }
 
 }  // namespace qsa

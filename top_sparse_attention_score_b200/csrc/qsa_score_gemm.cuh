@@ -20,7 +20,7 @@
 //     tile into a double-buffered shared stage in the 128-byte-swizzled layout,
 //     and the stores move whole 128-byte row segments to global memory;  TMEM holds two 256-column accumulators, so
 //     the epilogue of tile i overlaps the MMAs of tile i + 1;
-//   * every wait on an mbarrier is bounded (one second of %globaltimer): on
+//   * every wait on an mbarrier is bounded (four seconds of %globaltimer): on
 //     expiry the CTA records QSA_ERR_TIMEOUT in `status`, every role stops,
 //     in-flight copies and MMAs are drained (again with a bound) and TMEM is freed.
 #pragma once
@@ -277,7 +277,7 @@ __global__ void wait_selftest_kernel(uint32_t* status) {
     mbar_init(&gb.drain, 1);
     gb.abort = 0u;
     mbar_init_fence();
-    mbar_wait(&gb.drain, 0, &gb.abort, status);
+    mbar_wait(&gb.drain, 0, &gb.abort, status, kSelftestLimitNs);
   }
 }
 

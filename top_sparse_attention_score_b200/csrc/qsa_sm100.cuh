@@ -1,11 +1,14 @@
 // qsa_sm100.cuh -- sm_100a building blocks: mbarriers with bounded waits, TMA,
 // tcgen05 MMA / TMEM access and the shared-memory operand descriptors.
 //
-// Every wait on an mbarrier is bounded by one second of %globaltimer.  When a
+// Every wait on an mbarrier is bounded by %globaltimer: four seconds in the
+// step kernels (a healthy wait lasts microseconds; the margin covers a GPU
+// time-sliced with other processes), one second in the self-test.  When a
 // wait runs out, the waiting thread records QSA_ERR_TIMEOUT in the status word
 // and raises the CTA's abort flag; every other wait of the CTA then returns
 // false at once, so all roles leave their loops, drain what they issued and
-// reach the final barrier.
+// reach the final barrier.  The calls are asynchronous, so a caller learns of a
+// timeout only from qsa_device_status.
 #pragma once
 
 #include <cuda.h>
@@ -14,7 +17,8 @@
 
 namespace qsa {
 
-constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // one second
+constexpr unsigned long long kWaitLimitNs = 4000000000ull;      // step kernels: four seconds
+constexpr unsigned long long kSelftestLimitNs = 1000000000ull;  // the self-test: one second
 constexpr uint32_t kStatusTimeout = 4;                       // QSA_ERR_TIMEOUT
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -70,14 +74,15 @@ __device__ __forceinline__ bool mbar_try(uint32_t addr, uint32_t parity) {
 
 // Wait for the phase of `bar` with parity `parity`.  Returns false if the CTA
 // is aborting or the wait exceeded its limit (which starts the abort).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* abort, uint32_t* status) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* abort, uint32_t* status,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   const uint32_t addr = smem_u32(bar);
   if (mbar_try<false>(addr, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (;;) {
     if (*reinterpret_cast<volatile uint32_t*>(abort)) return false;
     if (mbar_try<false>(addr, parity)) return true;
-    if (global_ns() - t0 > kWaitLimitNs) {
+    if (global_ns() - t0 > limit_ns) {
       atomicExch(status, kStatusTimeout);
       *reinterpret_cast<volatile uint32_t*>(abort) = 1u;
       return false;

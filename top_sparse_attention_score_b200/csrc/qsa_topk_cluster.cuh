@@ -5,15 +5,16 @@
 // zipping, ...", what changed, item 1), organised around Blackwell clusters for the
 // latency of a decode step:
 //
-//   * a cluster of 8 CTAs x 512 threads owns one row; CTA r holds the order-
+//   * a cluster of 8 CTAs x 512 threads (16 CTAs for rows of more than 65536
+//     cells) owns one row; CTA r holds the order-
 //     preserving keys of cells [r * chunk, (r + 1) * chunk), read once from L2/HBM,
-//     and their coarse bins (the top 10 bits of the key of the score's fp16
+//     and their coarse bins (the top 12 bits of the key of the score's fp16
 //     rounding, so a higher bin always means a strictly larger score);
 //   * each CTA counts its bins in shared memory (two 16-bit counts per word);
 //     after one cluster barrier every CTA sums all eight through distributed
 //     shared memory and finds the threshold bin itself;
-//   * each CTA lists its cells in the threshold bin (typically a few hundred in
-//     the row); after a second barrier every CTA gathers all lists and one warp
+//   * each CTA lists its cells in the threshold bin (typically one to two hundred
+//     in the row); after a second barrier every CTA gathers all lists and one warp
 //     finds the exact k-th key over the bits the candidates do not share: up to
 //     1024 candidates held in registers, one bit per step, otherwise 8-bit digits
 //     counted in shared memory; it derives every CTA's output offset from the
@@ -34,19 +35,13 @@
 
 namespace qsa {
 
-constexpr int kClusterCtas = 8;
+constexpr int kClusterCtas = 8;         // CTAs per row up to 65536 cells
+constexpr int kClusterCtasWide = 16;    // CTAs per row up to 262144 cells (a non-portable cluster size)
 constexpr int kClusterThreads = 512;
-constexpr int kClusterRegPer = 16;       // keys per thread kept in registers; beyond, in shared memory
-constexpr int kClusterBins = 1024;       // coarse bins of the cluster histogram
+constexpr int kClusterRegPer = 32;       // keys per thread (registers): rows of up to 16 x 512 x 32 cells
+constexpr int kClusterBins = 4096;       // coarse bins of the cluster histogram (top 12 bits of score_key16)
 constexpr int kClusterCandCap = 2048;    // candidates one CTA can list
 constexpr int kClusterGatherCap = 4096;  // candidates a CTA can gather from the whole cluster
-
-// Coarse bin of an order-preserving key (score_key): the top 10 bits of the
-// order-preserving key of the score's fp16 rounding.
-__device__ __forceinline__ uint32_t cluster_bin(uint32_t key) {
-  const uint32_t bits = (key & 0x80000000u) ? (key ^ 0x80000000u) : ~key;
-  return score_bin(__uint_as_float(bits)) >> 1;
-}
 
 // One warp, 256 bins counted from the highest: the bin where the running count
 // first reaches k, and the count strictly above it (returned in every lane).
@@ -93,10 +88,10 @@ constexpr int kWarpSelSlots = 32;  // candidates per lane the register select ho
 // search ends early once a single candidate is left on the prefix: its key is
 // the answer.  Returns the key in `thr` and, in `take`, how many candidates
 // equal to it are kept (need minus the candidates above it).  The candidates of
-// CTA q are the gathered range [q_off[q], q_off[q + 1]); lanes q < kClusterCtas
+// CTA q are the gathered range [q_off[q], q_off[q + 1]); lanes q < C
 // set q_sel[q] = q_sure[q] + (those above thr) and q_eq[q] = (those equal to
 // thr) from per-slot ballot words staged in words[0, 64).
-template <int S>
+template <int S, int C>
 __device__ __forceinline__ void warp_select_regs(const uint32_t* gkey, const uint32_t* q_off, uint32_t n,
                                                  uint32_t need, const uint32_t* q_sure, uint32_t* q_sel,
                                                  uint32_t* q_eq, uint32_t* words, uint32_t& thr, uint32_t& take) {
@@ -162,8 +157,8 @@ __device__ __forceinline__ void warp_select_regs(const uint32_t* gkey, const uin
   words[lane] = w_gt;
   words[32 + lane] = w_eq;
   __syncwarp();
-  if (lane < static_cast<uint32_t>(kClusterCtas)) {
-    const uint32_t a = q_off[lane], b = lane + 1u < static_cast<uint32_t>(kClusterCtas) ? q_off[lane + 1] : n;
+  if (lane < static_cast<uint32_t>(C)) {
+    const uint32_t a = q_off[lane], b = lane + 1u < static_cast<uint32_t>(C) ? q_off[lane + 1] : n;
     uint32_t cg = 0u, ce = 0u;
     for (uint32_t w = a >> 5; a < b && w <= (b - 1u) >> 5; ++w) {
       const uint32_t lo = max(a, w * 32u) - w * 32u, hi = min(b, w * 32u + 32u) - w * 32u;
@@ -185,7 +180,7 @@ __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
 }
 
-template <int PER>
+template <int PER, int C>
 struct ClusterSmem {
   static constexpr int kWords = kClusterThreads * PER / 32;
   uint32_t hist[kClusterBins / 2];    // two 16-bit counts per word
@@ -198,56 +193,62 @@ struct ClusterSmem {
   uint32_t radix[2][256];
   uint32_t tmp256[256];
   uint32_t pub[4];                    // published: sure count, candidate count, selected count, tie count
-  uint32_t q_sure[kClusterCtas], q_cand[kClusterCtas], q_sel[kClusterCtas], q_eq[kClusterCtas];
-  uint32_t q_off[kClusterCtas];
+  uint32_t q_sure[C], q_cand[C], q_sel[C], q_eq[C];
+  uint32_t q_off[C];
   uint32_t cand_n, sure_n, misc[4];
   uint32_t scratch[33];
   uint32_t result[2];
 };
 
-template <int PER>
+template <int PER, int C>
 constexpr size_t cluster_smem_bytes() {
-  return sizeof(ClusterSmem<PER>) + (PER > kClusterRegPer ? static_cast<size_t>(PER) * kClusterThreads * 4 : 0);
+  return sizeof(ClusterSmem<PER, C>);
 }
 
-// grid (8, rows), cluster (8, 1, 1), block 512, dynamic smem cluster_smem_bytes<PER>().
-// PER cells per thread: the cluster covers 8 * 512 * PER cells, at least the longest row.
-template <int PER>
-__global__ void __launch_bounds__(kClusterThreads) cluster_select_kernel(const float* __restrict__ scores,
-                                                                         int64_t ld, int vis0, int top_k,
-                                                                         int32_t* __restrict__ ids) {
+// The selection of row blockIdx.y by this CTA of its C-CTA cluster (512 threads, shared
+// memory csm_raw of cluster_smem_bytes<PER, C>()): writes the row's ids, and when `list`
+// is not NULL also this CTA's own selected cells, ascending, to list[0 .. *list_n) (the
+// row's ids from position *list_at on).  On return every CTA of the cluster has finished
+// reading this CTA's shared memory.
+template <int PER, int C>
+__device__ __forceinline__ void cluster_select_row(const float* __restrict__ scores, int64_t ld, int vis0,
+                                                   int top_k, int32_t* __restrict__ ids, unsigned char* csm_raw,
+                                                   int* list, int* list_n, int* list_at) {
   namespace cg = cooperative_groups;
-  constexpr bool kInSmem = PER > kClusterRegPer;
+  static_assert(PER <= kClusterRegPer, "keys are held in registers");
   constexpr int NT = kClusterThreads;
   constexpr int CHUNK = NT * PER;
   constexpr int WORDS = CHUNK / 32;
-  extern __shared__ __align__(16) unsigned char csm_raw[];
-  ClusterSmem<PER>& sm = *reinterpret_cast<ClusterSmem<PER>*>(csm_raw);
-  uint32_t* skeys = reinterpret_cast<uint32_t*>(csm_raw + sizeof(ClusterSmem<PER>));
+  ClusterSmem<PER, C>& sm = *reinterpret_cast<ClusterSmem<PER, C>*>(csm_raw);
 
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
   const int tid = threadIdx.x;
   const int lane = tid & 31;
-  griddep_launch();
-  griddep_wait();
   const int row = blockIdx.y;
   const int V = vis0 + row;
   int32_t* out = ids + static_cast<size_t>(row) * top_k;
   if (V <= top_k) {  // every visible cell, ascending (the whole cluster leaves together)
     if (rank == 0)
       for (int i = tid; i < top_k; i += NT) out[i] = i < V ? i : -1;
+    if (list) {  // this CTA's share: cells [rank * CHUNK, ...) below V
+      const int lo = min(V, rank * CHUNK), hi = min(V, lo + CHUNK);
+      for (int i = tid; i < hi - lo; i += NT) list[i] = lo + i;
+      if (tid == 0) {
+        *list_n = hi - lo;
+        *list_at = lo;
+      }
+    }
     return;
   }
   const int c0 = rank * CHUNK;
   const float* s = scores + row * ld;
 
   // ---- keys of this CTA's cells (element e of thread t is cell c0 + e * NT + t)
-  uint32_t key[kInSmem ? 1 : PER];
-  uint32_t binpk[kInSmem ? 1 : (PER + 1) / 2];
-#define QSA_KEY(e) (kInSmem ? skeys[(e) * NT + tid] : key[kInSmem ? 0 : (e)])
-#define QSA_BIN(e) \
-  (kInSmem ? cluster_bin(QSA_KEY(e)) : ((binpk[kInSmem ? 0 : (e) >> 1] >> (16 * ((e) & 1))) & 0xffffu))
+  uint32_t key[PER];
+  uint32_t binpk[(PER + 1) / 2];
+#define QSA_KEY(e) (key[(e)])
+#define QSA_BIN(e) ((binpk[(e) >> 1] >> (16 * ((e) & 1))) & 0xffffu)
   {
     float x[PER];
 #pragma unroll
@@ -257,15 +258,10 @@ __global__ void __launch_bounds__(kClusterThreads) cluster_select_kernel(const f
     }
 #pragma unroll
     for (int e = 0; e < PER; ++e) {
-      const uint32_t k = score_key(x[e]);
-      if constexpr (kInSmem) {
-        skeys[e * NT + tid] = k;
-      } else {
-        key[e] = k;
-        const uint32_t b = score_bin(x[e]) >> 1;
-        if (e & 1) binpk[e >> 1] |= b << 16;
-        else binpk[e >> 1] = b;
-      }
+      key[e] = score_key(x[e]);
+      const uint32_t b = score_key16(x[e]) >> 4;
+      if (e & 1) binpk[e >> 1] |= b << 16;
+      else binpk[e >> 1] = b;
     }
   }
   for (int i = tid; i < kClusterBins / 2; i += NT) sm.hist[i] = 0u;
@@ -282,17 +278,21 @@ __global__ void __launch_bounds__(kClusterThreads) cluster_select_kernel(const f
     }
   cluster.sync();  // (1) every CTA's histogram is complete
 
-  // ---- every CTA: the row's histogram (one remote word per CTA and thread) and threshold bin
-  {
+  // ---- every CTA: the row's histogram (remote words of every CTA) and threshold bin
+#pragma unroll
+  for (int i = 0; i < kClusterBins / 2 / NT; ++i) {
+    const int wi = tid + i * NT;
+    uint32_t w[C];
+#pragma unroll
+    for (int q = 0; q < C; ++q) w[q] = cluster.map_shared_rank(sm.hist, q)[wi];
     uint32_t lo = 0u, hi = 0u;
 #pragma unroll
-    for (int q = 0; q < kClusterCtas; ++q) {
-      const uint32_t w = cluster.map_shared_rank(sm.hist, q)[tid];
-      lo += w & 0xffffu;
-      hi += w >> 16;
+    for (int q = 0; q < C; ++q) {
+      lo += w[q] & 0xffffu;
+      hi += w[q] >> 16;
     }
-    sm.tot[2 * tid] = lo;
-    sm.tot[2 * tid + 1] = hi;
+    sm.tot[2 * wi] = lo;
+    sm.tot[2 * wi + 1] = hi;
   }
   __syncthreads();
   uint32_t thr_bin, above;
@@ -338,7 +338,7 @@ __global__ void __launch_bounds__(kClusterThreads) cluster_select_kernel(const f
   }
   cluster.sync();  // (2) lists and counts published
 
-  if (tid < kClusterCtas) {
+  if (tid < C) {
     const uint32_t* p = cluster.map_shared_rank(sm.pub, tid);
     sm.q_sure[tid] = p[0];
     sm.q_cand[tid] = p[1];
@@ -347,7 +347,7 @@ __global__ void __launch_bounds__(kClusterThreads) cluster_select_kernel(const f
   uint32_t total_cand = 0u;
   bool fast = true;
 #pragma unroll
-  for (int q = 0; q < kClusterCtas; ++q) {
+  for (int q = 0; q < C; ++q) {
     if (tid == 0) sm.q_off[q] = total_cand;
     total_cand += sm.q_cand[q];
     fast = fast && sm.q_cand[q] <= static_cast<uint32_t>(kClusterCandCap);
@@ -360,7 +360,7 @@ __global__ void __launch_bounds__(kClusterThreads) cluster_select_kernel(const f
   if (fast) {
     // gather every candidate of the row; this CTA reads no remote memory after it
     for (uint32_t i = tid; i < total_cand; i += NT) {
-      int q = kClusterCtas - 1;
+      int q = C - 1;
       while (q > 0 && sm.q_off[q] > i) --q;
       const uint2 p = cluster.map_shared_rank(sm.cand, q)[i - sm.q_off[q]];
       sm.gkey[i] = p.x;
@@ -371,11 +371,11 @@ __global__ void __launch_bounds__(kClusterThreads) cluster_select_kernel(const f
     if (tid < 32 && total_cand <= 32u * kWarpSelSlots) {
       uint32_t pf, nd;
       if (total_cand <= 256u)
-        warp_select_regs<8>(sm.gkey, sm.q_off, total_cand, need, sm.q_sure, sm.q_sel, sm.q_eq, sm.tmp256, pf, nd);
+        warp_select_regs<8, C>(sm.gkey, sm.q_off, total_cand, need, sm.q_sure, sm.q_sel, sm.q_eq, sm.tmp256, pf, nd);
       else if (total_cand <= 512u)
-        warp_select_regs<16>(sm.gkey, sm.q_off, total_cand, need, sm.q_sure, sm.q_sel, sm.q_eq, sm.tmp256, pf, nd);
+        warp_select_regs<16, C>(sm.gkey, sm.q_off, total_cand, need, sm.q_sure, sm.q_sel, sm.q_eq, sm.tmp256, pf, nd);
       else
-        warp_select_regs<kWarpSelSlots>(sm.gkey, sm.q_off, total_cand, need, sm.q_sure, sm.q_sel, sm.q_eq,
+        warp_select_regs<kWarpSelSlots, C>(sm.gkey, sm.q_off, total_cand, need, sm.q_sure, sm.q_sel, sm.q_eq,
                                         sm.tmp256, pf, nd);
       if (lane == 0) {
         sm.misc[2] = pf;
@@ -413,7 +413,7 @@ __global__ void __launch_bounds__(kClusterThreads) cluster_select_kernel(const f
         mk |= wm << shift;
         top = shift - 1;
       }
-      if (lane < kClusterCtas) {
+      if (lane < C) {
         sm.q_sel[lane] = sm.q_sure[lane];
         sm.q_eq[lane] = 0u;
       }
@@ -450,7 +450,7 @@ __global__ void __launch_bounds__(kClusterThreads) cluster_select_kernel(const f
       if (tid < 256) {
         uint32_t sum = 0u;
 #pragma unroll
-        for (int q = 0; q < kClusterCtas; ++q) sum += cluster.map_shared_rank(h, q)[tid];
+        for (int q = 0; q < C; ++q) sum += cluster.map_shared_rank(h, q)[tid];
         sm.tmp256[tid] = sum;
       }
       __syncthreads();
@@ -510,7 +510,7 @@ __global__ void __launch_bounds__(kClusterThreads) cluster_select_kernel(const f
       sm.pub[3] = tot_eq;
     }
     cluster.sync();
-    if (tid < kClusterCtas) {
+    if (tid < C) {
       const uint32_t* p = cluster.map_shared_rank(sm.pub, tid);
       sm.q_sel[tid] = p[2];
       sm.q_eq[tid] = p[3];
@@ -544,13 +544,33 @@ __global__ void __launch_bounds__(kClusterThreads) cluster_select_kernel(const f
     while (b) {
       const int bit = __ffs(b) - 1;
       b &= b - 1u;
-      if (pos < static_cast<uint32_t>(top_k)) out[pos] = c0 + i * 32 + bit;
+      if (pos < static_cast<uint32_t>(top_k)) {
+        out[pos] = c0 + i * 32 + bit;
+        if (list) list[pos - out_before] = c0 + i * 32 + bit;
+      }
       ++pos;
     }
+  }
+  if (list && tid == 0) {
+    *list_n = static_cast<int>(min(tot_sel + my_take, static_cast<uint32_t>(top_k) - min(out_before, static_cast<uint32_t>(top_k))));
+    *list_at = static_cast<int>(out_before);
   }
   cluster_wait();  // every CTA has finished reading this CTA's shared memory
 #undef QSA_KEY
 #undef QSA_BIN
+}
+
+// grid (C, rows), cluster (C, 1, 1), block 512, dynamic smem cluster_smem_bytes<PER, C>().
+// PER cells per thread (held in registers): the cluster covers C * 512 * PER cells, at least
+// the longest row.
+template <int PER, int C>
+__global__ void __launch_bounds__(kClusterThreads) cluster_select_kernel(const float* __restrict__ scores,
+                                                                         int64_t ld, int vis0, int top_k,
+                                                                         int32_t* __restrict__ ids) {
+  extern __shared__ __align__(16) unsigned char csm_raw[];
+  griddep_launch();
+  griddep_wait();
+  cluster_select_row<PER, C>(scores, ld, vis0, top_k, ids, csm_raw, nullptr, nullptr, nullptr);
 }
 
 }  // namespace qsa

@@ -32,16 +32,18 @@ _F = ctypes.c_float
 SIGNATURES = {
     "qsa_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
     "qsa_cache_write": (_I, [_P, _I, _I, _P, _P, _P, _P]),
-    "qsa_decode": (_I, [_P, _I, _I, _P, _P, _P, _I, _I, _F, _P, _SZ, _P, _P, _P]),
-    "qsa_prefill_chunk": (_I, [_P, _I, _I, _P, _P, _P, _I, _F, _P, _SZ, _P, _P, _P]),
+    "qsa_decode": (_I, [_P, _I, _I, _P, _P, _P, _P, _P, _I, _I, _F, _P, _SZ, _P, _P, _P]),
+    "qsa_prefill_chunk": (_I, [_P, _I, _I, _P, _P, _P, _P, _P, _I, _F, _P, _SZ, _P, _P, _P]),
     "qsa_index_score": (_I, [_P, _I, _I, _P, _P, _P, _I64, _P]),
     "qsa_topk_workspace_bytes": (_SZ, [_I, _I, _I]),
     "qsa_topk": (_I, [_P, _I64, _I, _I, _I, _P, _SZ, _P, _P]),
-    "qsa_attn": (_I, [_P, _I, _P, _P, _I, _I, _F, _P, _P, _P]),
-    "qsa_merge": (_I, [_P, _I, _I, _P, _P]),
+    "qsa_attn": (_I, [_P, _I, _P, _P, _I, _I, _F, _P, _P, _P, _P]),
+    "qsa_merge": (_I, [_P, _I, _I, _P, _P, _P]),
     "qsa_topk_static": (_I, [_P, _I64, _I, _I, _I, _P, _P]),
     "qsa_device_status": (_I, [_P, _P]),
     "qsa_selftest_wait_timeout": (_I, [_P]),
+    "qsa_trace_begin": (_I, [_I, _P]),
+    "qsa_trace_end": (_I, [_I, _P, _P, _P]),
     "qsa_last_error": (ctypes.c_char_p, []),
     "qsa_launch_count": (ctypes.c_uint64, []),
 }
@@ -56,6 +58,25 @@ class QSAError(RuntimeError):
 class CacheStruct(ctypes.Structure):
     _fields_ = [("k", _P), ("v", _P), ("ks", _P), ("vs", _P), ("idx_key", _P),
                 ("max_cells", ctypes.c_int32)]
+
+
+class NewCellsStruct(ctypes.Structure):
+    """qsa_new_cells: the step's own cells, appended by the step call itself."""
+    _fields_ = [("k", _P), ("v", _P), ("idx_key", _P)]
+
+
+def _new_cells(append, rows):
+    """(struct, reference to keep alive) for append = (k, v, key) tensors, or (None, None)."""
+    if append is None:
+        return None, None
+    k, v, key = append
+    for t, name in ((k, "append k"), (v, "append v")):
+        _dev(t, torch.float32, name)
+        if t.shape[0] != rows:
+            raise ValueError(f"{name} has {t.shape[0]} rows, the call has {rows}")
+    _dev(key, torch.float16, "append idx_key")
+    st = NewCellsStruct(k.data_ptr(), v.data_ptr(), key.data_ptr())
+    return ctypes.byref(st), st
 
 
 _lib = None
@@ -177,34 +198,43 @@ def cache_write(cache: DeviceCache, pos0: int, k, v, key, stream=None) -> None:
                                   _ptr(_dev(key, torch.float16, "key")), _stream(stream)))
 
 
+def _opt(t, dtype, name):
+    return None if t is None else _ptr(_dev(t, dtype, name))
+
+
 def decode(cache: DeviceCache, L: int, q, iq, iw, top_k: int, nsplit: int = 0, scale: float = 1 / 16,
-           ws=None, out=None, ids_out=None, stream=None):
+           ws=None, out=None, ids_out=None, stream=None, append=None, gate=None):
+    """One decode step of n = q.shape[0] tokens.  append = (k, v, idx_key) writes the
+    tokens' own cells at L - n .. L - 1 first (in the same call); gate multiplies the
+    output by sigmoid(gate)."""
     n = q.shape[0]
     if ws is None:
         ws = workspace(workspace_bytes(MODE_DECODE, n, L, top_k, nsplit), q.device)
     if out is None:
         out = torch.empty(n, HQ, D, dtype=torch.float32, device=q.device)
-    _check(load().qsa_decode(cache.ref(), L, n, _ptr(_dev(q, torch.float32, "q")),
+    app, _keep = _new_cells(append, n)
+    _check(load().qsa_decode(cache.ref(), L, n, app, _ptr(_dev(q, torch.float32, "q")),
                              _ptr(_dev(iq, torch.float16, "iq")), _ptr(_dev(iw, torch.float32, "iw")),
-                             top_k, nsplit, scale, _ptr(ws), ws.numel(), _ptr(out),
-                             _ptr(None if ids_out is None else _dev(ids_out, torch.int32, "ids_out")),
-                             _stream(stream)))
+                             _opt(gate, torch.float32, "gate"), top_k, nsplit, scale, _ptr(ws), ws.numel(),
+                             _ptr(out), _opt(ids_out, torch.int32, "ids_out"), _stream(stream)))
     return out
 
 
 def prefill_chunk(cache: DeviceCache, pos0: int, q, iq, iw, top_k: int, scale: float = 1 / 16,
-                  ws=None, out=None, ids_out=None, stream=None):
+                  ws=None, out=None, ids_out=None, stream=None, append=None, gate=None):
+    """One prompt chunk of T = q.shape[0] tokens at pos0.  append = (k, v, idx_key) writes
+    the chunk's cells at pos0 .. pos0 + T - 1 first (in the same call)."""
     T = q.shape[0]
     if ws is None:
         ws = workspace(workspace_bytes(MODE_PREFILL, T, pos0 + T, top_k), q.device)
     if out is None:
         out = torch.empty(T, HQ, D, dtype=torch.float32, device=q.device)
-    _check(load().qsa_prefill_chunk(cache.ref(), pos0, T, _ptr(_dev(q, torch.float32, "q")),
+    app, _keep = _new_cells(append, T)
+    _check(load().qsa_prefill_chunk(cache.ref(), pos0, T, app, _ptr(_dev(q, torch.float32, "q")),
                                     _ptr(_dev(iq, torch.float16, "iq")),
-                                    _ptr(_dev(iw, torch.float32, "iw")), top_k, scale, _ptr(ws),
-                                    ws.numel(), _ptr(out),
-                                    _ptr(None if ids_out is None else _dev(ids_out, torch.int32, "ids_out")),
-                                    _stream(stream)))
+                                    _ptr(_dev(iw, torch.float32, "iw")), _opt(gate, torch.float32, "gate"),
+                                    top_k, scale, _ptr(ws), ws.numel(), _ptr(out),
+                                    _opt(ids_out, torch.int32, "ids_out"), _stream(stream)))
     return out
 
 
@@ -232,25 +262,52 @@ def topk(scores, vis0: int, top_k: int, ws=None, ids=None, stream=None):
 
 
 def attn(cache: DeviceCache, q, ids, nsplit: int = 1, scale: float = 1 / 16, part=None, out=None,
-         stream=None):
+         stream=None, gate=None):
     rows, top_k = ids.shape
     if nsplit == 1 and out is None:
         out = torch.empty(rows, HQ, D, dtype=torch.float32, device=q.device)
     if nsplit > 1 and part is None:
         part = torch.empty(rows, HQ, nsplit, PART_STRIDE, dtype=torch.float32, device=q.device)
     _check(load().qsa_attn(cache.ref(), rows, _ptr(_dev(q, torch.float32, "q")),
-                           _ptr(_dev(ids, torch.int32, "ids")), top_k, nsplit, scale, _ptr(part),
-                           _ptr(out), _stream(stream)))
+                           _ptr(_dev(ids, torch.int32, "ids")), top_k, nsplit, scale,
+                           _opt(gate, torch.float32, "gate"), _ptr(part), _ptr(out), _stream(stream)))
     return out if nsplit == 1 else part
 
 
-def merge(part, out=None, stream=None):
+def merge(part, out=None, stream=None, gate=None):
     rows, _, nsplit, _ = part.shape
     if out is None:
         out = torch.empty(rows, HQ, D, dtype=torch.float32, device=part.device)
     _check(load().qsa_merge(_ptr(_dev(part, torch.float32, "part")), rows, nsplit,
-                            _ptr(_dev(out, torch.float32, "out")), _stream(stream)))
+                            _opt(gate, torch.float32, "gate"), _ptr(_dev(out, torch.float32, "out")),
+                            _stream(stream)))
     return out
+
+
+class trace:
+    """Per-kernel device times of the library calls made inside the block, on one stream:
+
+        with qsa.trace() as t:
+            qsa.decode(...)
+        t.kernels  ->  [(name, ms), ...]
+
+    Events between the kernels serialise them; the times are those of back-to-back kernels.
+    """
+
+    def __init__(self, capacity: int = 256, stream=None):
+        self.capacity, self.stream, self.kernels = capacity, stream, []
+
+    def __enter__(self):
+        _check(load().qsa_trace_begin(self.capacity, _stream(self.stream)))
+        return self
+
+    def __exit__(self, *exc):
+        n = ctypes.c_int(0)
+        ms = (ctypes.c_float * self.capacity)()
+        names = (ctypes.c_char_p * self.capacity)()
+        _check(load().qsa_trace_end(self.capacity, ctypes.byref(n), ms, names))
+        self.kernels = [(names[i].decode(), float(ms[i])) for i in range(min(n.value, self.capacity))]
+        return False
 
 
 def device_status(stream=None) -> int:
