@@ -428,6 +428,15 @@ def test_decode_config1(gpu, n):
     _decode_case(gpu, synth.make_workload(1, n=n))
 
 
+@pytest.mark.parametrize("n", [1, 3])
+def test_decode_long_rows_auto_split(gpu, n):
+    # rows of more than 65536 cells with the automatic split: one 16-CTA selection cluster
+    # per row, then 32 pieces of attention and their merge
+    wl = synth.make_workload(2, n=n)
+    wl.nsplit = 0
+    _decode_case(gpu, wl)
+
+
 def test_decode_config2(gpu):
     _decode_case(gpu, synth.make_workload(2))
 
@@ -517,7 +526,7 @@ def test_decode_nsplit_invariance(gpu):
     wl = synth.make_workload(1, n=2, cells=6000)
     cache, q, iq, iw = dev_inputs(qsa, wl)
     outs, idss = [], []
-    for ns in (1, 2, 7, 64):
+    for ns in (1, 2, 7, 64, 0):  # 0: the automatic split
         ids = torch.empty(2, wl.top_k, dtype=torch.int32, device=DEV)
         outs.append(qsa.decode(cache, wl.L, q, iq, iw, wl.top_k, ns, wl.scale, ids_out=ids).cpu().numpy())
         idss.append(ids.cpu().numpy())

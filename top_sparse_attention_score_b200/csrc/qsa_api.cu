@@ -145,6 +145,7 @@ int prepare_device() {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(qsa::cluster_select_kernel<32, qsa::kClusterCtasWide>,
                              cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(qsa::score_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              qsa::kGemmSmemRequest);

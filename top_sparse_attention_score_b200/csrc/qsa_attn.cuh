@@ -80,7 +80,7 @@ __device__ __forceinline__ int attn_cell(const int* rid, int dv, int p, int end)
   else return __ldg(rid + p);
 }
 
-// ---- pieces shared by attn_kernel and the fused decode kernel
+// ---- the pieces of attn_kernel
 
 // Online-softmax state of one W-warp group for one (row, KV head): the reference
 // maximum (log2 units) of P, finite from the start so a block with no valid cell gives

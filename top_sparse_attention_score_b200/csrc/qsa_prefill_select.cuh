@@ -387,40 +387,74 @@ __global__ void __launch_bounds__(kSsThreads, 1)
         break;
       }
       tc_fence_after();
-      uint32_t rr[4][16];
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        tmem_ld16(tmem + (static_cast<uint32_t>(quad * 32) << 16) +
-                      static_cast<uint32_t>(buf * kSsN + 64 * cq + 16 * c),
-                  rr[c]);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar.acc_empty[buf]);  // the accumulator is in registers
       const int cell = ct * kSsCells + quad * 32 + lane;
       uint32_t* seg_cnt = cnt + seg * kSsTokens;
+      // Scores of the warp's 32 cells for its 16 tokens (two TMEM loads of 8 tokens x 4
+      // heads), two tokens at a time in packed fp32 (the same fma chain per token): lane tl
+      // keeps token tl's ballot of candidates, every lane the set of tokens its cell is a
+      // candidate of.
+      float sc[16];
+      uint32_t my_hits = 0u, mine = 0u;
+      uint32_t rr[2][16];
 #pragma unroll
-      for (int tl = 0; tl < 16; ++tl) {
-        const float4 wv = *reinterpret_cast<const float4*>(tab + tl * kSsTable);
-        const float thr = tab[tl * kSsTable + 4];
-        const int V = __float_as_int(tab[tl * kSsTable + 5]);
-        const uint32_t* d = &rr[tl >> 2][(tl & 3) * 4];
-        float sc = wv.x * fmaxf(__uint_as_float(d[0]), 0.f);
-        sc = fmaf(wv.y, fmaxf(__uint_as_float(d[1]), 0.f), sc);
-        sc = fmaf(wv.z, fmaxf(__uint_as_float(d[2]), 0.f), sc);
-        sc = fmaf(wv.w, fmaxf(__uint_as_float(d[3]), 0.f), sc);
-        // the warp's candidates of this token: one shared-memory atomic per warp
-        const bool hit = cell < V && sc >= thr;
-        const uint32_t m = __ballot_sync(0xffffffffu, hit);
-        if (m) {
-          uint32_t base = 0u;
-          if (lane == 0) base = atomicAdd(&seg_cnt[16 * cq + tl], static_cast<uint32_t>(__popc(m)));
-          base = __shfl_sync(0xffffffffu, base, 0);
-          const uint32_t slot = base + __popc(m & ((1u << lane) - 1u));
-          if (hit && slot < static_cast<uint32_t>(cap)) {
-            const size_t lb = (static_cast<size_t>(__float_as_uint(tab[tl * kSsTable + 7])) << 32) |
-                              __float_as_uint(tab[tl * kSsTable + 6]);
-            a.cand[lb + slot] = make_uint2(score_key(sc), static_cast<uint32_t>(cell));
+      for (int tp = 0; tp < 8; ++tp) {
+        if ((tp & 3) == 0) {  // columns of tokens 2 tp .. 2 tp + 7
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+            tmem_ld16(tmem + (static_cast<uint32_t>(quad * 32) << 16) +
+                          static_cast<uint32_t>(buf * kSsN + 64 * cq + 16 * (2 * (tp >> 2) + c)),
+                      rr[c]);
+          tmem_ld_wait();
+          if (tp == 4) {  // the accumulator is in registers: hand it back to the MMA warp
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar.acc_empty[buf]);
+          }
+        }
+        const int ta = 2 * tp, tb2 = ta + 1;
+        const float4 wa = *reinterpret_cast<const float4*>(tab + ta * kSsTable);
+        const float4 wb = *reinterpret_cast<const float4*>(tab + tb2 * kSsTable);
+        const uint32_t* da = &rr[(ta >> 2) & 1][(ta & 3) * 4];
+        const uint32_t* db = &rr[(tb2 >> 2) & 1][(tb2 & 3) * 4];
+        float2 x = __fmul2_rn(make_float2(wa.x, wb.x), make_float2(fmaxf(__uint_as_float(da[0]), 0.f),
+                                                                   fmaxf(__uint_as_float(db[0]), 0.f)));
+        x = __ffma2_rn(make_float2(wa.y, wb.y),
+                       make_float2(fmaxf(__uint_as_float(da[1]), 0.f), fmaxf(__uint_as_float(db[1]), 0.f)), x);
+        x = __ffma2_rn(make_float2(wa.z, wb.z),
+                       make_float2(fmaxf(__uint_as_float(da[2]), 0.f), fmaxf(__uint_as_float(db[2]), 0.f)), x);
+        x = __ffma2_rn(make_float2(wa.w, wb.w),
+                       make_float2(fmaxf(__uint_as_float(da[3]), 0.f), fmaxf(__uint_as_float(db[3]), 0.f)), x);
+        sc[ta] = x.x;
+        sc[tb2] = x.y;
+        const float2 ta_tv = *reinterpret_cast<const float2*>(tab + ta * kSsTable + 4);   // threshold, V
+        const float2 tb_tv = *reinterpret_cast<const float2*>(tab + tb2 * kSsTable + 4);
+        const bool ha = cell < __float_as_int(ta_tv.y) && x.x >= ta_tv.x;
+        const bool hb = cell < __float_as_int(tb_tv.y) && x.y >= tb_tv.x;
+        const uint32_t ma = __ballot_sync(0xffffffffu, ha), mb = __ballot_sync(0xffffffffu, hb);
+        my_hits = lane == ta ? ma : (lane == tb2 ? mb : my_hits);
+        mine |= (ha ? 1u : 0u) << ta;
+        mine |= (hb ? 1u : 0u) << tb2;
+      }
+      // one round of shared-memory atomics reserves every token's slots
+      uint32_t my_base = 0u;
+      if (lane < 16 && my_hits) my_base = atomicAdd(&seg_cnt[16 * cq + lane], static_cast<uint32_t>(__popc(my_hits)));
+      const uint32_t below = (1u << lane) - 1u;
+      // each lane writes its own candidates, one token per step (as many steps as the most
+      // any lane has)
+      while (__any_sync(0xffffffffu, mine != 0u)) {
+        const int tl = mine ? __ffs(mine) - 1 : 0;
+        const uint32_t m = __shfl_sync(0xffffffffu, my_hits, tl);
+        const uint32_t base = __shfl_sync(0xffffffffu, my_base, tl);
+        if (mine) {
+          mine &= mine - 1u;
+          const uint32_t slot = base + __popc(m & below);
+          if (slot < static_cast<uint32_t>(cap)) {
+            float v = sc[0];
+#pragma unroll
+            for (int j2 = 1; j2 < 16; ++j2) v = tl == j2 ? sc[j2] : v;
+            const uint2 lb2 = *reinterpret_cast<const uint2*>(tab + tl * kSsTable + 6);
+            const size_t lb = (static_cast<size_t>(lb2.y) << 32) | lb2.x;
+            a.cand[lb + slot] = make_uint2(score_key(v), static_cast<uint32_t>(cell));
           }
         }
       }

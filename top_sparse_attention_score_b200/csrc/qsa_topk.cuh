@@ -7,8 +7,7 @@
 // Radix select spread over many SMs, with no CTA ever waiting on another:
 //   histogram  2048-bin count of each score's coarse bin (top 11 bits of the
 //              order-preserving key of its fp16 rounding), accumulated in shared
-//              memory and flushed with atomics -- either fused into the decode
-//              score kernel or by topk_hist_kernel.  The CTA that finishes last
+//              memory and flushed with atomics by topk_hist_kernel.  The CTA that finishes last
 //              (a fence and a counter, no waiting) finds each row's threshold bin.
 //   filter     topk_filter_kernel: each CTA appends the cells of its chunk above
 //              the threshold bin to the row's "sure" list and the cells in it, with

@@ -201,19 +201,16 @@ struct ClusterSmem {
 };
 
 template <int PER, int C>
-constexpr size_t cluster_smem_bytes() {
+__host__ __device__ constexpr size_t cluster_smem_bytes() {
   return sizeof(ClusterSmem<PER, C>);
 }
 
 // The selection of row blockIdx.y by this CTA of its C-CTA cluster (512 threads, shared
-// memory csm_raw of cluster_smem_bytes<PER, C>()): writes the row's ids, and when `list`
-// is not NULL also this CTA's own selected cells, ascending, to list[0 .. *list_n) (the
-// row's ids from position *list_at on).  On return every CTA of the cluster has finished
-// reading this CTA's shared memory.
+// memory csm_raw of cluster_smem_bytes<PER, C>()): writes the row's ids.  On return every
+// CTA of the cluster has finished reading this CTA's shared memory.
 template <int PER, int C>
 __device__ __forceinline__ void cluster_select_row(const float* __restrict__ scores, int64_t ld, int vis0,
-                                                   int top_k, int32_t* __restrict__ ids, unsigned char* csm_raw,
-                                                   int* list, int* list_n, int* list_at) {
+                                                   int top_k, int32_t* __restrict__ ids, unsigned char* csm_raw) {
   namespace cg = cooperative_groups;
   static_assert(PER <= kClusterRegPer, "keys are held in registers");
   constexpr int NT = kClusterThreads;
@@ -231,14 +228,6 @@ __device__ __forceinline__ void cluster_select_row(const float* __restrict__ sco
   if (V <= top_k) {  // every visible cell, ascending (the whole cluster leaves together)
     if (rank == 0)
       for (int i = tid; i < top_k; i += NT) out[i] = i < V ? i : -1;
-    if (list) {  // this CTA's share: cells [rank * CHUNK, ...) below V
-      const int lo = min(V, rank * CHUNK), hi = min(V, lo + CHUNK);
-      for (int i = tid; i < hi - lo; i += NT) list[i] = lo + i;
-      if (tid == 0) {
-        *list_n = hi - lo;
-        *list_at = lo;
-      }
-    }
     return;
   }
   const int c0 = rank * CHUNK;
@@ -544,16 +533,9 @@ __device__ __forceinline__ void cluster_select_row(const float* __restrict__ sco
     while (b) {
       const int bit = __ffs(b) - 1;
       b &= b - 1u;
-      if (pos < static_cast<uint32_t>(top_k)) {
-        out[pos] = c0 + i * 32 + bit;
-        if (list) list[pos - out_before] = c0 + i * 32 + bit;
-      }
+      if (pos < static_cast<uint32_t>(top_k)) out[pos] = c0 + i * 32 + bit;
       ++pos;
     }
-  }
-  if (list && tid == 0) {
-    *list_n = static_cast<int>(min(tot_sel + my_take, static_cast<uint32_t>(top_k) - min(out_before, static_cast<uint32_t>(top_k))));
-    *list_at = static_cast<int>(out_before);
   }
   cluster_wait();  // every CTA has finished reading this CTA's shared memory
 #undef QSA_KEY
@@ -570,7 +552,7 @@ __global__ void __launch_bounds__(kClusterThreads) cluster_select_kernel(const f
   extern __shared__ __align__(16) unsigned char csm_raw[];
   griddep_launch();
   griddep_wait();
-  cluster_select_row<PER, C>(scores, ld, vis0, top_k, ids, csm_raw, nullptr, nullptr, nullptr);
+  cluster_select_row<PER, C>(scores, ld, vis0, top_k, ids, csm_raw);
 }
 
 }  // namespace qsa
