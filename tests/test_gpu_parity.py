@@ -365,6 +365,47 @@ def test_attn_single_and_empty(gpu):
     assert np.all(np.isneginf(part[1, :, :, 0])) and np.all(part[1, :, :, 1:] == 0)
 
 
+@pytest.mark.parametrize("rows,k", [(9, 1), (12, 300), (17, 4096)])
+def test_attn_prompt_kernel_edges(gpu, rows, k):
+    # more than 8 rows in one piece (the prompt-chunk kernel): lists shorter than one
+    # 32-cell block, ragged last blocks, an empty row, ids past the cache as empty slots,
+    # a query head of zeros (equal weights), the output gate in the epilogue
+    qsa = gpu
+    cells = 5000
+    cache_h = synth.make_cache(231, cells)
+    q, _, _ = synth.make_queries(232, rows)
+    q[2, 5] = 0.0
+    nvalid = [k, 0] + [max(1, (k * (r + 1)) // rows) for r in range(rows - 2)]
+    ids = _id_lists(233, rows, cells, k, nvalid)
+    if k > 1:
+        ids[0, -1] = cells + 7
+    gate = _gate(234, rows)
+    cache = qsa.DeviceCache.from_host(cache_h, DEV)
+    out = qsa.attn(cache, torch.from_numpy(q).to(DEV), torch.from_numpy(ids).to(DEV), 1, 1 / 16,
+                   gate=gate).cpu().numpy()
+    g = gate.cpu().numpy()
+    assert np.all(out[1] == 0)  # no cells at all
+    for r in [0] + list(range(2, rows)):
+        ids_r = np.where((ids[r] >= 0) & (ids[r] < cells), ids[r], -1).astype(np.int32)
+        ref = oracle.gate_row(oracle.attn_row(cache_h, q[r], ids_r, 1 / 16), g[r])
+        assert rel_err(out[r], ref) <= OUT_TOL, f"row {r}"
+
+
+def test_attn_prompt_kernel_golden(gpu):
+    # the hand-worked softmax fixture as ten rows of one call (the prompt-chunk kernel)
+    from tests import pins
+    qsa = gpu
+    cache_h, q, vals, _ = pins.softmax_golden_case()
+    cache = qsa.DeviceCache.from_host(cache_h, DEV)
+    dims = 2.0 ** -(np.arange(256) // 32)
+    want = np.stack([vals["out"][h // 12] * dims for h in range(24)])
+    ids = torch.arange(4, dtype=torch.int32, device=DEV)[None].repeat(10, 1)
+    qd = torch.from_numpy(np.repeat(q[None], 10, 0)).to(DEV)
+    out = qsa.attn(cache, qd, ids, 1, 1 / 16).cpu().numpy()
+    for r in range(10):
+        assert rel_err(out[r], want) <= OUT_TOL
+
+
 def test_merge_vs_oracle(gpu):
     qsa = gpu
     st = synth.Stream(301, "merge")
