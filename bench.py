@@ -507,7 +507,8 @@ def kernel_times(qsa, torch, w, spec, stream, reps):
     """Average device time of every kernel the step's calls launch, per launch, from the
     library's own trace events (qsa_trace_begin / qsa_trace_end) around the real calls."""
     acc, count = {}, {}
-    info = {"union_cells": 0, "rows": 0, "cells_scored": 0, "ncells": 0, "nsplit": {}, "calls": 0}
+    info = {"union_cells": 0, "gathered_cells": 0, "rows": 0, "cells_scored": 0, "ncells": 0, "nsplit": {},
+            "calls": 0}
     ids = torch.empty(max(spec.ns), spec.top_k, dtype=torch.int32, device=w.out.device)
     # Each call sits behind a ~1.5 ms torch sleep kernel so the host has queued all of its
     # launches before the first starts: the events bracket kernels, not launch gaps.
@@ -532,6 +533,7 @@ def kernel_times(qsa, torch, w, spec, stream, reps):
                 ncells = spec.L if spec.kind == "decode" else spec.pos0 + spec.T
                 idn = ids[:n].cpu().numpy()
                 info["union_cells"] += int(np.unique(idn[idn >= 0]).size)
+                info["gathered_cells"] += int((idn >= 0).sum())
                 info["rows"] += n
                 info["cells_scored"] += int(sum(vis0 + r for r in range(n)))
                 info["ncells"] += ncells * n
@@ -600,6 +602,12 @@ def roofline(spec, kern, pk):
               "new cells: fp32 K/V and fp16 keys read, int8 codes, fp16 scales and keys written")
     hbm_entry("attn_kernel", attn_bytes, "union of the rows' selected cells x 1088 B + q, ids, out"
               + (" (prefill: gathered from L2 mostly)" if spec.kind == "prefill" else ""))
+    if "attn_kernel" in kernels and spec.kind == "prefill":
+        # every (row, selected cell) gathers 1088 B (both KV heads' codes and scales), most of it
+        # from L2: the rate the prompt-chunk attention sustains on its gathers
+        gathered = info["gathered_cells"] / calls * CELL_BYTES
+        kernels["attn_kernel"]["gathered_bytes_per_launch"] = gathered
+        kernels["attn_kernel"]["gather_gbs"] = gathered / (kernels["attn_kernel"]["ms"] / 1e3) / 1e9
     if "merge_kernel" in avg:
         ns = info["nsplit"]
         part_bytes = sum(n * 24 * ns[n] * 258 * 4 + n * 24 * 256 * 4 for n in ns) / calls
