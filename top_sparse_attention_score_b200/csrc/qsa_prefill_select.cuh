@@ -44,7 +44,8 @@ constexpr int kSsCapPerTile = 16;    // candidate slots per (token, cell tile) o
 constexpr int kSsCapSlack = 64;
 constexpr int kSsTable = 8;          // words per token of an epilogue warp's table
 constexpr int kSsSmemBytes = kSsQBytes + kSsStages * kSsKeyBytes + kSsEpiWarps * 16 * kSsTable * 4 +
-                             2 * kSsTokens * 4 + 512 /*barriers*/ + 1024 /*align*/;
+                             2 * kSsTokens * 4 + kSsEpiWarps * 16 * 32 * 4 /*scores*/ +
+                             kSsEpiWarps * 16 * 4 /*ballots*/ + 512 /*barriers*/ + 1024 /*align*/;
 static_assert(kSsSmemBytes > 114 * 1024, "one GEMM CTA per SM (it allocates all 512 TMEM columns)");
 constexpr int kPfThreads = 512;      // final kernel (two CTAs per SM)
 constexpr int kPfCand = 8192;        // candidates a final CTA holds in shared memory
@@ -239,7 +240,9 @@ __global__ void __launch_bounds__(kSsThreads, 1)
   unsigned char* sK = base + kSsQBytes;                      // stages x 128 cells x 128 B
   float* table = reinterpret_cast<float*>(sK + kSsStages * kSsKeyBytes);  // [16 warps][16 tokens][8]
   uint32_t* cnt = reinterpret_cast<uint32_t*>(table + kSsEpiWarps * 16 * kSsTable);  // [2][64]
-  SsBarriers& bar = *reinterpret_cast<SsBarriers*>(cnt + 2 * kSsTokens);
+  float* stage = reinterpret_cast<float*>(cnt + 2 * kSsTokens);  // [16 warps][16 tokens][32 lanes] scores
+  uint32_t* ballots = reinterpret_cast<uint32_t*>(stage + kSsEpiWarps * 16 * 32);  // [16 warps][16 tokens]
+  SsBarriers& bar = *reinterpret_cast<SsBarriers*>(ballots + kSsEpiWarps * 16);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x;
@@ -348,6 +351,8 @@ __global__ void __launch_bounds__(kSsThreads, 1)
     const int quad = warp & 3;            // TMEM lanes 32 quad .. + 31: this warp's cells
     const int cq = e >> 2;                // columns 64 cq .. + 63: tokens 16 cq .. + 15 of the block
     float* tab = table + e * 16 * kSsTable;
+    float* stw = stage + e * 16 * 32;  // this warp's scores, [token][lane]
+    uint32_t* balw = ballots + e * 16;  // this warp's ballots, [token]
     int cur_tb = -1, li = 0;
     bool ok = true;
     for (int it = it0; it < it1 && ok; ++it) {
@@ -390,11 +395,11 @@ __global__ void __launch_bounds__(kSsThreads, 1)
       const int cell = ct * kSsCells + quad * 32 + lane;
       uint32_t* seg_cnt = cnt + seg * kSsTokens;
       // Scores of the warp's 32 cells for its 16 tokens (two TMEM loads of 8 tokens x 4
-      // heads), two tokens at a time in packed fp32 (the same fma chain per token): lane tl
-      // keeps token tl's ballot of candidates, every lane the set of tokens its cell is a
-      // candidate of.
-      float sc[16];
-      uint32_t my_hits = 0u, mine = 0u;
+      // heads), two tokens at a time in packed fp32 (the same fma chain per token), staged in
+      // shared memory for the candidate writes; each token's ballot of candidates goes to
+      // shared memory too (lane t reads token t's), every lane keeps the set of tokens its
+      // cell is a candidate of.
+      uint32_t mine = 0u;
       uint32_t rr[2][16];
 #pragma unroll
       for (int tp = 0; tp < 8; ++tp) {
@@ -424,17 +429,22 @@ __global__ void __launch_bounds__(kSsThreads, 1)
                        make_float2(fmaxf(__uint_as_float(da[2]), 0.f), fmaxf(__uint_as_float(db[2]), 0.f)), x);
         x = __ffma2_rn(make_float2(wa.w, wb.w),
                        make_float2(fmaxf(__uint_as_float(da[3]), 0.f), fmaxf(__uint_as_float(db[3]), 0.f)), x);
-        sc[ta] = x.x;
-        sc[tb2] = x.y;
+        stw[ta * 32 + lane] = x.x;
+        stw[tb2 * 32 + lane] = x.y;
         const float2 ta_tv = *reinterpret_cast<const float2*>(tab + ta * kSsTable + 4);   // threshold, V
         const float2 tb_tv = *reinterpret_cast<const float2*>(tab + tb2 * kSsTable + 4);
         const bool ha = cell < __float_as_int(ta_tv.y) && x.x >= ta_tv.x;
         const bool hb = cell < __float_as_int(tb_tv.y) && x.y >= tb_tv.x;
         const uint32_t ma = __ballot_sync(0xffffffffu, ha), mb = __ballot_sync(0xffffffffu, hb);
-        my_hits = lane == ta ? ma : (lane == tb2 ? mb : my_hits);
+        if (lane == 0) {
+          balw[ta] = ma;
+          balw[tb2] = mb;
+        }
         mine |= (ha ? 1u : 0u) << ta;
         mine |= (hb ? 1u : 0u) << tb2;
       }
+      __syncwarp();
+      const uint32_t my_hits = lane < 16 ? balw[lane] : 0u;
       // one round of shared-memory atomics reserves every token's slots
       uint32_t my_base = 0u;
       if (lane < 16 && my_hits) my_base = atomicAdd(&seg_cnt[16 * cq + lane], static_cast<uint32_t>(__popc(my_hits)));
@@ -449,9 +459,7 @@ __global__ void __launch_bounds__(kSsThreads, 1)
           mine &= mine - 1u;
           const uint32_t slot = base + __popc(m & below);
           if (slot < static_cast<uint32_t>(cap)) {
-            float v = sc[0];
-#pragma unroll
-            for (int j2 = 1; j2 < 16; ++j2) v = tl == j2 ? sc[j2] : v;
+            const float v = stw[tl * 32 + lane];
             const uint2 lb2 = *reinterpret_cast<const uint2*>(tab + tl * kSsTable + 6);
             const size_t lb = (static_cast<size_t>(lb2.y) << 32) | lb2.x;
             a.cand[lb + slot] = make_uint2(score_key(v), static_cast<uint32_t>(cell));
