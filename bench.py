@@ -335,30 +335,36 @@ class Workload:
         self.h_buf, hv = _packed(torch, host, pin=True)
         for view, a in zip(hv, host):
             view.copy_(torch.from_numpy(a))
-        self.d_buf, (self.q, self.iq, self.iw, self.kn, self.vn, self.keyn) = _packed(torch, host, dev)
-        self.d_buf.copy_(self.h_buf)
+        # two device sets of inputs and outputs (and two pinned output buffers), so the
+        # end-to-end run copies one step's data while the neighbouring step computes
         self.out_rows = sum(spec.ns)
-        self.out = torch.empty(self.out_rows, 24, 256, dtype=torch.float32, device=dev)
-        self.out_h = torch.empty(self.out.shape, dtype=torch.float32).pin_memory()
+        self.d_bufs, self.call_sets, self.outs, self.outs_h = [], [], [], []
+        for _ in range(2):
+            d_buf, (q, iq, iw, kn, vn, keyn) = _packed(torch, host, dev)
+            d_buf.copy_(self.h_buf)
+            out = torch.empty(self.out_rows, 24, 256, dtype=torch.float32, device=dev)
+            calls, at = [], 0
+            for n in spec.ns:  # each call's views, made once (a caller with fixed buffers holds them)
+                calls.append((n, q[:n], iq[:n], iw[:n], (kn[:n], vn[:n], keyn[:n]), out[at:at + n]))
+                at += n
+            self.d_bufs.append(d_buf)
+            self.call_sets.append(calls)
+            self.outs.append(out)
+            self.outs_h.append(torch.empty(out.shape, dtype=torch.float32).pin_memory())
+        self.calls, self.out = self.call_sets[0], self.outs[0]
         if spec.kind == "decode":
             nbytes = max(qsa.workspace_bytes(qsa.MODE_DECODE, n, spec.L, spec.top_k, spec.nsplit) for n in spec.ns)
         else:
             nbytes = qsa.workspace_bytes(qsa.MODE_PREFILL, spec.T, spec.pos0 + spec.T, spec.top_k)
         self.ws = qsa.workspace(nbytes, dev)
-        # each call's views, made once (a caller with fixed buffers holds them)
-        self.calls, at = [], 0
-        for n in spec.ns:
-            self.calls.append((n, self.q[:n], self.iq[:n], self.iw[:n],
-                               (self.kn[:n], self.vn[:n], self.keyn[:n]), self.out[at:at + n]))
-            at += n
         self.h2d_bytes = int(self.h_buf.numel())
         self.d2h_bytes = int(self.out.numel() * 4)
 
-    def step(self, qsa, i):
+    def step(self, qsa, i, b=0):
         """One step: every call of the workload through the public API, each appending
-        its rows' own cells in the same call (cache copy i % ROTATE)."""
+        its rows' own cells in the same call (cache copy i % ROTATE, input and output set b)."""
         spec, c = self.spec, self.caches[i % ROTATE]
-        for n, q, iq, iw, app, out in self.calls:
+        for n, q, iq, iw, app, out in self.call_sets[b]:
             if spec.kind == "decode":
                 qsa.decode(c, spec.L, q, iq, iw, spec.top_k, spec.nsplit, self.wl.scale, ws=self.ws, out=out,
                            append=app)
@@ -417,17 +423,55 @@ def measure(torch, qsa, spec, args, dev, stream, world, local, with_cpu):
         g.reset()
     del graphs
 
-    # ---- end to end through the public API: one copy of the packed inputs from pinned host
-    # memory, the calls (each appending its rows' cells), one copy of all outputs back
-    def e2e_step(i):
-        w.d_buf.copy_(w.h_buf, non_blocking=True)
-        w.step(qsa, i)
-        w.out_h.copy_(w.out, non_blocking=True)
+    # ---- end to end through the public API: per step one copy of the packed inputs from
+    # pinned host memory, the calls (each appending its rows' cells), one copy of all outputs
+    # back into pinned host memory.  The copies run on two copy streams (in and out) with two
+    # input / output sets, so step i + 1's inputs arrive and step i - 1's outputs leave while
+    # step i computes; every copy of every step is inside the timed region.
+    cs_in, cs_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev_h2d, ev_comp, ev_d2h = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
 
-    for i in range(2):
-        e2e_step(i)
-    e2e_times = [timed_pass(steps, e2e_step) for _ in range(3)]
+    def e2e_pass(k):
+        barrier(world)
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        cs_in.wait_event(ev0)
+        cs_out.wait_event(ev0)
+        for i in range(k):
+            b = i & 1
+            with torch.cuda.stream(cs_in):
+                if i >= 2:
+                    cs_in.wait_event(ev_comp[b])  # step i - 2 has read this input set
+                w.d_bufs[b].copy_(w.h_buf, non_blocking=True)
+                ev_h2d[b].record(cs_in)
+            stream.wait_event(ev_h2d[b])
+            if i >= 2:
+                stream.wait_event(ev_d2h[b])  # step i - 2's outputs have left this output set
+            w.step(qsa, i, b)
+            ev_comp[b].record(stream)
+            with torch.cuda.stream(cs_out):
+                cs_out.wait_event(ev_comp[b])
+                w.outs_h[b].copy_(w.outs[b], non_blocking=True)
+                ev_d2h[b].record(cs_out)
+        for b in range(min(k, 2)):
+            stream.wait_event(ev_d2h[b])
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        return ev0.elapsed_time(ev1)
+
+    e2e_pass(4)
+    e2e_times = [e2e_pass(steps) for _ in range(3)]
     e2e_value, _ = job_rate(spec.units, steps, statistics.median(e2e_times), world)
+
+    # the same with each step's copies and calls back to back on one stream (no overlap)
+    def serial_step(i):
+        w.d_bufs[0].copy_(w.h_buf, non_blocking=True)
+        w.step(qsa, i, 0)
+        w.outs_h[0].copy_(w.outs[0], non_blocking=True)
+
+    timed_pass(2, serial_step)
+    serial_times = [timed_pass(steps, serial_step) for _ in range(3)]
+    serial_value, _ = job_rate(spec.units, steps, statistics.median(serial_times), world)
 
     # ---- per-kernel durations, step-level calls with events on the same stream
     kern = kernel_times(qsa, torch, w, spec, stream, 20)
@@ -441,9 +485,12 @@ def measure(torch, qsa, spec, args, dev, stream, world, local, with_cpu):
                             f"({ROTATE * spec.L * (CELL_BYTES + KEY_BYTES) / 1e6:.0f} MB > 126 MB L2)",
                       "timing": f"median of {passes} passes of {steps} graph-replayed steps"},
            "e2e": {"value": e2e_value, "unit": spec.unit, "h2d_bytes_per_step": w.h2d_bytes,
-                   "d2h_bytes_per_step": w.d2h_bytes,
-                   "api": "one H2D copy of the packed inputs, one call per row group appending its "
-                          "cells (qsa_decode / qsa_prefill_chunk with append), one D2H copy of the outputs"},
+                   "d2h_bytes_per_step": w.d2h_bytes, "serial_value": serial_value,
+                   "api": "per step one H2D copy of the packed inputs from pinned memory, one call per row "
+                          "group appending its cells (qsa_decode / qsa_prefill_chunk with append), one D2H "
+                          "copy of the outputs to pinned memory; copies on an input and an output copy stream, "
+                          "double-buffered, overlapping the neighbouring steps' calls (serial_value: copies and "
+                          "calls of each step back to back on one stream)"},
            "gpu_launches": per_graph * steps,
            "roofline": roof["main"], "kernels": roof["kernels"], "clocks": clk.summary()}
     if "score_attn" in roof:
