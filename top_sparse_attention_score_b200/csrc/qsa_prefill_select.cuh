@@ -173,14 +173,20 @@ __global__ void __launch_bounds__(kPsThreads) prefill_threshold_kernel(PrefillSe
   const int vmax = a.vis0 + rb + nrows - 1;               // cells the block's last row sees
   const int R = max(kPsStride, (vmax + kPsSamples - 1) / kPsSamples);  // sample stride
   const int ns = (vmax + R - 1) / R;                      // sampled cells j * R < vmax
-  for (int base = warp * 16; base < ns; base += (kPsThreads / 32) * 16) {
+  constexpr int kStep = (kPsThreads / 32) * 16;  // samples the CTA's warps take per round
+  auto key = [&](int s) {
+    return s < ns ? reinterpret_cast<const uint4*>(a.keys + static_cast<size_t>(s) * R * kDI) : nullptr;
+  };
+  // the keys of the next two rounds are in flight while one round is scored
+  GemvKeys K0 = gemv_load_keys(key(warp * 16 + g), key(warp * 16 + g + 8));
+  GemvKeys K1 = gemv_load_keys(key(warp * 16 + kStep + g), key(warp * 16 + kStep + g + 8));
+  for (int base = warp * 16; base < ns; base += kStep) {
     const int s0 = base + g, s1 = base + g + 8;
-    const uint4* k0 = s0 < ns ? reinterpret_cast<const uint4*>(a.keys + static_cast<size_t>(s0) * R * kDI)
-                              : nullptr;
-    const uint4* k1 = s1 < ns ? reinterpret_cast<const uint4*>(a.keys + static_cast<size_t>(s1) * R * kDI)
-                              : nullptr;
+    const GemvKeys K2 = gemv_load_keys(key(base + 2 * kStep + g), key(base + 2 * kStep + g + 8));
     float sc[4];
-    gemv_scores(Q, k0, k1, w, nj, sc);
+    gemv_mma(Q, K0, w, nj, sc);
+    K0 = K1;
+    K1 = K2;
     const int slot = (t & 1) ? s1 : s0;
     const int cell = slot * R;
 #pragma unroll
