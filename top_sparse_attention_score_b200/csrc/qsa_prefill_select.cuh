@@ -658,12 +658,26 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_final_kernel(PrefillSel
   if (!s_bad) {
     // ---- the candidates: load, select exactly, emit in index order
     const int n = static_cast<int>(seg_off[nseg]);
-    for (int i = tid; i < n; i += NT) {
-      int s = 0;
-      while (seg_off[s + 1] <= static_cast<uint32_t>(i)) ++s;
-      const uint2 p = __ldcg(a.cand + seg_base[s] + (i - seg_off[s]));
-      ckey[i] = p.x;
-      ccell[i] = p.y;
+    constexpr int kBatch = 8;  // loads in flight per thread before their stores
+    for (int i0 = tid; i0 < n; i0 += NT * kBatch) {
+      uint2 p[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int i = i0 + u * NT;
+        if (i < n) {
+          int s = 0;
+          while (seg_off[s + 1] <= static_cast<uint32_t>(i)) ++s;
+          p[u] = __ldcg(a.cand + seg_base[s] + (i - seg_off[s]));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int i = i0 + u * NT;
+        if (i < n) {
+          ckey[i] = p[u].x;
+          ccell[i] = p[u].y;
+        }
+      }
     }
     __syncthreads();
     smem_radix_select<NT>(ckey, n, static_cast<uint32_t>(a.top_k), sm, thr_key, take_eq);
