@@ -137,16 +137,34 @@ __device__ __forceinline__ void attn_load_q(uint32_t (&aq)[kNG / W][2][4], const
     }
 }
 
-// Gather one block of 32 cells into `st` with NT threads (tid = 0 .. NT - 1): slot i holds
-// cell cell_of(i), an empty slot for one < 0 or >= max_cells.
+// The cells one thread gathers of a 32-cell block: chunk u (K and V rows) is cell
+// (tid + NT u) / 16, the scales' cell is tid % 32 (for tid < 64).
+template <int NT>
+struct AttnIds {
+  static constexpr int kChunks = 512 / NT;
+  int chunk[kChunks];
+  int scale;
+};
+
+// The ids of one block (cell_of(i): list slot i), loaded a block before its gather.
 template <int NT, class CellOf>
-__device__ __forceinline__ void attn_gather(AttnStage& st, const AttnArgs& a, int kvh, int tid, CellOf cell_of) {
+__device__ __forceinline__ void attn_load_ids(AttnIds<NT>& ids, int tid, CellOf cell_of) {
+#pragma unroll
+  for (int u = 0; u < AttnIds<NT>::kChunks; ++u) ids.chunk[u] = cell_of((tid + NT * u) >> 4);
+  ids.scale = tid < 2 * kAttnCells ? cell_of(tid & 31) : -1;
+}
+
+// Gather one block of 32 cells into `st` with NT threads (tid = 0 .. NT - 1): slot i holds
+// the cell of ids, an empty slot for one < 0 or >= max_cells.
+template <int NT>
+__device__ __forceinline__ void attn_gather(AttnStage& st, const AttnArgs& a, int kvh, int tid,
+                                            const AttnIds<NT>& ids) {
   // K and V rows: 32 cells x 16 chunks of 16 bytes each, 512 / NT + 512 / NT per thread.
 #pragma unroll
-  for (int u = 0; u < 512 / NT; ++u) {
+  for (int u = 0; u < AttnIds<NT>::kChunks; ++u) {
     const int chunk = tid + NT * u;
     const int i = chunk >> 4, part = chunk & 15;
-    int cell = cell_of(i);
+    int cell = ids.chunk[u];
     const bool ok = cell >= 0 && cell < a.max_cells;
     if (!ok) cell = 0;
     const size_t row = (static_cast<size_t>(cell) * kHKV + kvh) * kD + part * 16;
@@ -155,7 +173,7 @@ __device__ __forceinline__ void attn_gather(AttnStage& st, const AttnArgs& a, in
   }
   if (tid < 2 * kAttnCells) {  // scales: 64 rows of 16 bytes
     const int i = tid & 31;
-    int cell = cell_of(i);
+    int cell = ids.scale;
     const bool ok = cell >= 0 && cell < a.max_cells;
     if (tid < kAttnCells) st.valid[i] = ok;
     if (!ok) cell = 0;
@@ -333,24 +351,29 @@ __global__ void __launch_bounds__(32 * W) attn_kernel(AttnArgs a) {
       for (int p = beg + static_cast<int>(threadIdx.x); p < end; p += NT)
         a.ids_fill[static_cast<size_t>(row) * a.top_k + p] = p < dv ? p : -1;
   }
-  auto gather = [&](int blk) {
+  // a block's ids are loaded one block before its gather is issued
+  AttnIds<NT> ids;
+  auto load_ids = [&](int blk) {
     const int p0 = beg + blk * kAttnCells;
-    attn_gather<NT>(sm.st[blk % kAttnStages], a, kvh, static_cast<int>(threadIdx.x),
-                    [&](int i) { return attn_cell<kAll>(rid, dv, p0 + i, end); });
+    attn_load_ids<NT>(ids, static_cast<int>(threadIdx.x),
+                      [&](int i) { return attn_cell<kAll>(rid, dv, p0 + i, end); });
   };
-#pragma unroll
-  for (int st = 0; st < kAttnStages - 1; ++st) {
-    if (st < nblk) gather(st);
-    cp_async_commit();
+  static_assert(kAttnStages == 2, "the id prefetch below assumes a double-buffered ring");
+  if (nblk > 0) {
+    load_ids(0);
+    attn_gather<NT>(sm.st[0], a, kvh, static_cast<int>(threadIdx.x), ids);
   }
+  cp_async_commit();
+  if (nblk > 1) load_ids(1);
 
   AttnState<W> S;
   S.init();
   for (int b = 0; b < nblk; ++b) {
     // refill the stage block b - 1 used (every warp finished it at the last barrier)
-    const int nb = b + kAttnStages - 1;
-    if (nb < nblk) gather(nb);
+    const int nb = b + 1;
+    if (nb < nblk) attn_gather<NT>(sm.st[nb % kAttnStages], a, kvh, static_cast<int>(threadIdx.x), ids);
     cp_async_commit();
+    if (nb + 1 < nblk) load_ids(nb + 1);
     cp_async_wait<kAttnStages - 1>();
     __syncthreads();
     attn_block<W>(sm.st[b % kAttnStages], sm.red, aq, S, warp, [] { __syncthreads(); });
