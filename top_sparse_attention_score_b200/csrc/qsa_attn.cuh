@@ -351,20 +351,22 @@ __global__ void __launch_bounds__(32 * W) attn_kernel(AttnArgs a) {
       for (int p = beg + static_cast<int>(threadIdx.x); p < end; p += NT)
         a.ids_fill[static_cast<size_t>(row) * a.top_k + p] = p < dv ? p : -1;
   }
-  // a block's ids are loaded one block before its gather is issued
+  // a block's ids are loaded one block before its gather is issued (the first two blocks'
+  // together, so the second gather does not wait for its ids)
   AttnIds<NT> ids;
-  auto load_ids = [&](int blk) {
+  auto load_ids = [&](AttnIds<NT>& dst, int blk) {
     const int p0 = beg + blk * kAttnCells;
-    attn_load_ids<NT>(ids, static_cast<int>(threadIdx.x),
+    attn_load_ids<NT>(dst, static_cast<int>(threadIdx.x),
                       [&](int i) { return attn_cell<kAll>(rid, dv, p0 + i, end); });
   };
   static_assert(kAttnStages == 2, "the id prefetch below assumes a double-buffered ring");
   if (nblk > 0) {
-    load_ids(0);
-    attn_gather<NT>(sm.st[0], a, kvh, static_cast<int>(threadIdx.x), ids);
+    AttnIds<NT> ids0;
+    load_ids(ids0, 0);
+    if (nblk > 1) load_ids(ids, 1);
+    attn_gather<NT>(sm.st[0], a, kvh, static_cast<int>(threadIdx.x), ids0);
   }
   cp_async_commit();
-  if (nblk > 1) load_ids(1);
 
   AttnState<W> S;
   S.init();
@@ -373,7 +375,7 @@ __global__ void __launch_bounds__(32 * W) attn_kernel(AttnArgs a) {
     const int nb = b + 1;
     if (nb < nblk) attn_gather<NT>(sm.st[nb % kAttnStages], a, kvh, static_cast<int>(threadIdx.x), ids);
     cp_async_commit();
-    if (nb + 1 < nblk) load_ids(nb + 1);
+    if (nb + 1 < nblk) load_ids(ids, nb + 1);
     cp_async_wait<kAttnStages - 1>();
     __syncthreads();
     attn_block<W>(sm.st[b % kAttnStages], sm.red, aq, S, warp, [] { __syncthreads(); });
