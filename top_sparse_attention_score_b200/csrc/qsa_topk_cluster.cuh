@@ -8,8 +8,9 @@
 //   * a cluster of 8 CTAs x 512 threads (16 CTAs for rows of more than 65536
 //     cells) owns one row; CTA r holds the order-
 //     preserving keys of cells [r * chunk, (r + 1) * chunk), read once from L2/HBM,
-//     and their coarse bins (the top 12 bits of the key of the score's fp16
-//     rounding, so a higher bin always means a strictly larger score);
+//     and their coarse bins (the top 11 bits of the key of the score's fp16
+//     rounding, so a higher bin always means a strictly larger score: 2048 bins,
+//     whose summed histogram every CTA reads from all the others);
 //   * each CTA counts its bins in shared memory (two 16-bit counts per word);
 //     after one cluster barrier every CTA sums all eight through distributed
 //     shared memory and finds the threshold bin itself;
@@ -39,7 +40,8 @@ constexpr int kClusterCtas = 8;         // CTAs per row up to 65536 cells
 constexpr int kClusterCtasWide = 16;    // CTAs per row up to 262144 cells (a non-portable cluster size)
 constexpr int kClusterThreads = 512;
 constexpr int kClusterRegPer = 32;       // keys per thread (registers): rows of up to 16 x 512 x 32 cells
-constexpr int kClusterBins = 4096;       // coarse bins of the cluster histogram (top 12 bits of score_key16)
+constexpr int kClusterBins = 2048;       // coarse bins of the cluster histogram (top 11 bits of score_key16)
+static_assert(kClusterBins / 2 % kClusterThreads == 0, "the histogram sum gives every thread whole words");
 constexpr int kClusterCandCap = 2048;    // candidates one CTA can list
 constexpr int kClusterGatherCap = 4096;  // candidates a CTA can gather from the whole cluster
 
@@ -248,7 +250,7 @@ __device__ __forceinline__ void cluster_select_row(const float* __restrict__ sco
 #pragma unroll
     for (int e = 0; e < PER; ++e) {
       key[e] = score_key(x[e]);
-      const uint32_t b = score_key16(x[e]) >> 4;
+      const uint32_t b = score_key16(x[e]) >> 5;
       if (e & 1) binpk[e >> 1] |= b << 16;
       else binpk[e >> 1] = b;
     }
