@@ -212,25 +212,30 @@ __global__ void __launch_bounds__(128) index_score_kernel(const __half* __restri
   const int groups = (ncells + kScoreCellsPerWarp - 1) / kScoreCellsPerWarp;
   const int step = score_ctas * kScoreWarps;
   int grp = blockIdx.x * kScoreWarps + warp;
-  GemvKeys K;
-  if (grp < groups) K = gemv_load_keys(key_row(grp * 16 + g), key_row(grp * 16 + g + 8));
+  // the keys of this warp's next two groups are in flight while one group is scored (rows of
+  // many cells give each warp several groups)
+  auto load = [&](int gr) {
+    GemvKeys K;
+    if (gr < groups) K = gemv_load_keys(key_row(gr * 16 + g), key_row(gr * 16 + g + 8));
+    return K;
+  };
+  GemvKeys K0 = load(grp), K1 = load(grp + step);
   __syncthreads();
   GemvQ Q;
   gemv_load_q(Q, s_iq);
   griddep_wait();
   for (; grp < groups; grp += step) {
-    const int nxt = grp + step;
-    GemvKeys Kn;
-    if (nxt < groups) Kn = gemv_load_keys(key_row(nxt * 16 + g), key_row(nxt * 16 + g + 8));
+    const GemvKeys K2 = load(grp + 2 * step);
     float sc[4];
-    gemv_mma(Q, K, w, nj, sc);
+    gemv_mma(Q, K0, w, nj, sc);
     const int c = grp * 16 + g + 8 * (t & 1);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int row = rb + 2 * j + (t >> 1);
       if (j < nj && row < rows && c < ncells) scores[row * ld + c] = sc[j];
     }
-    if (nxt < groups) K = Kn;
+    K0 = K1;
+    K1 = K2;
   }
 }
 
