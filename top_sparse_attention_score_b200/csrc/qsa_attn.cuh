@@ -42,6 +42,14 @@ struct __align__(16) AttnStage {
 };
 
 constexpr int kAttnStages = 2;
+
+// 2^x by the hardware approximation (ex2.approx.ftz: subnormal results flush to zero; the
+// weights it feeds are rounded to fp16 and never exceed 2^8, so nothing below 2^-126 matters).
+__device__ __forceinline__ float attn_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 constexpr float kAttnShift = 8.f;      // log2 margin before the reference maximum moves
 constexpr float kAttnNoMax = -1.0e30f;  // reference maximum before the first valid cell
 
@@ -261,7 +269,7 @@ __device__ __forceinline__ void attn_block(const AttnStage& st, float4 (*red)[4]
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
       const float mnew = fmaxf(S.m_run[r], mx[r]);
-      const float alpha = exp2f(S.m_run[r] - mnew);
+      const float alpha = attn_exp2(S.m_run[r] - mnew);
       S.l_run[r] *= alpha;
       S.m_run[r] = mnew;
 #pragma unroll
@@ -279,7 +287,7 @@ __device__ __forceinline__ void attn_block(const AttnStage& st, float4 (*red)[4]
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       const int r = c >> 1;
-      const float p = exp2f(s[nt][c] - S.m_run[r]);
+      const float p = attn_exp2(s[nt][c] - S.m_run[r]);
       s[nt][c] = p;
       rs[r] += p;
     }
@@ -412,7 +420,7 @@ __global__ void __launch_bounds__(32 * W) attn_kernel(AttnArgs a) {
         *reinterpret_cast<float4*>(dst) = lo;
         *reinterpret_cast<float4*>(dst + 4) = hi;
       } else {  // partials relative to the true maximum
-        const float corr = (S.m_top[r] == -INFINITY) ? 0.f : exp2f(S.m_run[r] - S.m_top[r]);
+        const float corr = (S.m_top[r] == -INFINITY) ? 0.f : attn_exp2(S.m_run[r] - S.m_top[r]);
         lo.x *= corr; lo.y *= corr; lo.z *= corr; lo.w *= corr;
         hi.x *= corr; hi.y *= corr; hi.z *= corr; hi.w *= corr;
         float* dst = a.part + (rh * a.nsplit + split) * kPart;
