@@ -162,6 +162,30 @@ __device__ __forceinline__ void attn_load_ids(AttnIds<NT>& ids, int tid, CellOf 
   ids.scale = tid < 2 * kAttnCells ? cell_of(tid & 31) : -1;
 }
 
+// The K codes enter the QK^T tiles as fp16 1152 + code (one byte-permute, no subtraction):
+// each group's accumulator starts at -1152 times the group's sum of fp16 q instead, for rows g
+// (kb[gi][0]) and g + 8 (kb[gi][1]).  The sums are of the fp16 fragments the MMAs read, over
+// the quad's 32 dims of the group.
+template <int W>
+__device__ __forceinline__ void attn_k_bias(float (&kb)[kNG / W][2], const uint32_t (&aq)[kNG / W][2][4]) {
+#pragma unroll
+  for (int gi = 0; gi < kNG / W; ++gi)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      float sum = 0.f;
+#pragma unroll
+      for (int s = 0; s < 2; ++s)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&aq[gi][s][r + 2 * h]));
+          sum += f.x + f.y;
+        }
+      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+      kb[gi][r] = -1152.f * sum;
+    }
+}
+
 // Gather one block of 32 cells into `st` with NT threads (tid = 0 .. NT - 1): slot i holds
 // the cell of ids, an empty slot for one < 0 or >= max_cells.
 template <int NT>
@@ -197,8 +221,8 @@ __device__ __forceinline__ void attn_gather(AttnStage& st, const AttnArgs& a, in
 // maximum, the weights and P.V into the warp's O.  `sync` is the group's barrier.
 template <int W, class Sync>
 __device__ __forceinline__ void attn_block(const AttnStage& st, float4 (*red)[4][32],
-                                           const uint32_t (&aq)[kNG / W][2][4], AttnState<W>& S, int warp,
-                                           Sync sync) {
+                                           const uint32_t (&aq)[kNG / W][2][4], const float (&kb)[kNG / W][2],
+                                           AttnState<W>& S, int warp, Sync sync) {
   constexpr int GW = kNG / W;
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const uint32_t valid = __ballot_sync(0xffffffffu, st.valid[lane] != 0);  // bit c: slot c holds a cell
@@ -215,9 +239,9 @@ __device__ __forceinline__ void attn_block(const AttnStage& st, float4 (*red)[4]
       const int qg = GW * warp + gi;
       const uint2 kw = *reinterpret_cast<const uint2*>(krow + 32 * qg + 8 * t);
       const uint32_t x0 = kw.x ^ 0x80808080u, x1 = kw.y ^ 0x80808080u;
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      mma_f16_16816(acc, aq[gi][0], i8x2_to_h2(x0, 0x4140u), i8x2_to_h2(x0, 0x4342u));
-      mma_f16_16816(acc, aq[gi][1], i8x2_to_h2(x1, 0x4140u), i8x2_to_h2(x1, 0x4342u));
+      float acc[4] = {kb[gi][0], kb[gi][0], kb[gi][1], kb[gi][1]};
+      mma_f16_16816(acc, aq[gi][0], i8x2_to_h2_biased(x0, 0x4140u), i8x2_to_h2_biased(x0, 0x4342u));
+      mma_f16_16816(acc, aq[gi][1], i8x2_to_h2_biased(x1, 0x4140u), i8x2_to_h2_biased(x1, 0x4342u));
       const float2 sc = make_float2(__half2float(st.ks[(8 * nt + 2 * t) * kNG + qg]),
                                     __half2float(st.ks[(8 * nt + 2 * t + 1) * kNG + qg]));
       s[nt][0] = fmaf(sc.x, acc[0], s[nt][0]);
@@ -318,10 +342,14 @@ __device__ __forceinline__ void attn_block(const AttnStage& st, float4 (*red)[4]
       const uint32_t wD = *reinterpret_cast<const uint32_t*>(vb + (cA + 9) * kAttnVStride) ^ 0x80808080u;
       const __half2 sAB = __halves2half2(st.vs[cA * kNG + qg], st.vs[(cA + 1) * kNG + qg]);
       const __half2 sCD = __halves2half2(st.vs[(cA + 8) * kNG + qg], st.vs[(cA + 9) * kNG + qg]);
+      // the two cells' bytes interleaved once: [A0 B0 A1 B1] and [A2 B2 A3 B3]
+      const uint32_t ab[2] = {__byte_perm(wA, wB, 0x5140u), __byte_perm(wA, wB, 0x7362u)};
+      const uint32_t cd[2] = {__byte_perm(wC, wD, 0x5140u), __byte_perm(wC, wD, 0x7362u)};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        uint32_t b0 = i8_pair_to_h2(wA, wB, i);
-        uint32_t b1 = i8_pair_to_h2(wC, wD, i);
+        const uint32_t sel = (i & 1) ? 0x4342u : 0x4140u;
+        uint32_t b0 = i8x2_to_h2(ab[i >> 1], sel);
+        uint32_t b1 = i8x2_to_h2(cd[i >> 1], sel);
         const __half2 h0 = __hmul2(*reinterpret_cast<const __half2*>(&b0), sAB);
         const __half2 h1 = __hmul2(*reinterpret_cast<const __half2*>(&b1), sCD);
         mma_f16_16816(S.o[gi][i], pa, *reinterpret_cast<const uint32_t*>(&h0),
@@ -351,6 +379,8 @@ __global__ void __launch_bounds__(32 * W) attn_kernel(AttnArgs a) {
 
   uint32_t aq[GW][2][4];
   attn_load_q<W>(aq, a.q + (static_cast<size_t>(row) * kHQ + kvh * kQPerKV) * kD, a.scale_log2, warp);
+  float kb[GW][2];
+  attn_k_bias<W>(kb, aq);
 
   // The ids come from the selection kernel: wait for it before the first gather.
   griddep_wait();
@@ -386,7 +416,7 @@ __global__ void __launch_bounds__(32 * W) attn_kernel(AttnArgs a) {
     if (nb + 1 < nblk) load_ids(ids, nb + 1);
     cp_async_wait<kAttnStages - 1>();
     __syncthreads();
-    attn_block<W>(sm.st[b % kAttnStages], sm.red, aq, S, warp, [] { __syncthreads(); });
+    attn_block<W>(sm.st[b % kAttnStages], sm.red, aq, kb, S, warp, [] { __syncthreads(); });
     __syncthreads();
   }
   cp_async_wait<0>();

@@ -46,10 +46,9 @@ __device__ __forceinline__ uint32_t i8x2_to_h2(uint32_t x, uint32_t sel) {
   return *reinterpret_cast<const uint32_t*>(&r);
 }
 
-// Byte i of xa and byte i of xb (both XORed with 0x80) -> fp16 pair (xa_i, xb_i).
-__device__ __forceinline__ uint32_t i8_pair_to_h2(uint32_t xa, uint32_t xb, int i) {
-  const uint32_t t = __byte_perm(xa, xb, static_cast<uint32_t>(i | ((i + 4) << 4)));
-  return i8x2_to_h2(t, 0x4140u);
+// The same two bytes as fp16 1152 + code (exact; the caller removes the 1152).
+__device__ __forceinline__ uint32_t i8x2_to_h2_biased(uint32_t x, uint32_t sel) {
+  return __byte_perm(x, 0x64646464u, sel);
 }
 
 // The output gate ("attention + gate"): the attention output is multiplied
