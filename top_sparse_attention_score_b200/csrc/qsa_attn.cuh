@@ -215,6 +215,25 @@ __device__ __forceinline__ void attn_gather(AttnStage& st, const AttnArgs& a, in
   }
 }
 
+// N consecutive fp16 scales (N = 2 or 4, 4N-byte aligned) as floats, in one shared load.
+template <int N>
+__device__ __forceinline__ void attn_load_scales(const __half* p, float (&f)[N]) {
+  if constexpr (N == 4) {
+    const uint2 w = *reinterpret_cast<const uint2*>(p);
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&w.x));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&w.y));
+    f[0] = a.x;
+    f[1] = a.y;
+    f[2] = b.x;
+    f[3] = b.y;
+  } else {
+    static_assert(N == 2, "two or four scales");
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(p));
+    f[0] = a.x;
+    f[1] = a.y;
+  }
+}
+
 // One gathered block through the online softmax, for warp `warp` of a W-warp group:
 // partial QK^T over the warp's dims, the group's partial scores summed through `red`
 // (every warp in the same order, so all agree bit for bit), masking, the running
@@ -234,6 +253,10 @@ __device__ __forceinline__ void attn_block(const AttnStage& st, float4 (*red)[4]
 #pragma unroll
     for (int c = 0; c < 4; ++c) s[nt][c] = 0.f;
     const int8_t* krow = st.k + (8 * nt + g) * kAttnKStride;
+    // the K scales of this warp's groups for cells 8 nt + 2t and 8 nt + 2t + 1, one load each
+    float ksa[GW], ksb[GW];
+    attn_load_scales<GW>(st.ks + (8 * nt + 2 * t) * kNG + GW * warp, ksa);
+    attn_load_scales<GW>(st.ks + (8 * nt + 2 * t + 1) * kNG + GW * warp, ksb);
 #pragma unroll
     for (int gi = 0; gi < GW; ++gi) {
       const int qg = GW * warp + gi;
@@ -242,8 +265,7 @@ __device__ __forceinline__ void attn_block(const AttnStage& st, float4 (*red)[4]
       float acc[4] = {kb[gi][0], kb[gi][0], kb[gi][1], kb[gi][1]};
       mma_f16_16816(acc, aq[gi][0], i8x2_to_h2_biased(x0, 0x4140u), i8x2_to_h2_biased(x0, 0x4342u));
       mma_f16_16816(acc, aq[gi][1], i8x2_to_h2_biased(x1, 0x4140u), i8x2_to_h2_biased(x1, 0x4342u));
-      const float2 sc = make_float2(__half2float(st.ks[(8 * nt + 2 * t) * kNG + qg]),
-                                    __half2float(st.ks[(8 * nt + 2 * t + 1) * kNG + qg]));
+      const float2 sc = make_float2(ksa[gi], ksb[gi]);
       s[nt][0] = fmaf(sc.x, acc[0], s[nt][0]);
       s[nt][1] = fmaf(sc.y, acc[1], s[nt][1]);
       s[nt][2] = fmaf(sc.x, acc[2], s[nt][2]);
@@ -331,6 +353,19 @@ __device__ __forceinline__ void attn_block(const AttnStage& st, float4 (*red)[4]
     pa[2] = pack_half2(s[2 * s2 + 1][0], s[2 * s2 + 1][1]);
     pa[3] = pack_half2(s[2 * s2 + 1][2], s[2 * s2 + 1][3]);
     const int cA = 16 * s2 + 2 * t;  // cells of k-index 2t, 2t+1, 2t+8, 2t+9
+    // their V scales for this warp's groups: one load per cell (two fp16 per word)
+    uint32_t vsw[4][(GW + 1) / 2];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const __half* p = st.vs + (cA + (k & 1) + 8 * (k >> 1)) * kNG + GW * warp;
+      if constexpr (GW == 4) {
+        const uint2 w = *reinterpret_cast<const uint2*>(p);
+        vsw[k][0] = w.x;
+        vsw[k][1] = w.y;
+      } else {
+        vsw[k][0] = *reinterpret_cast<const uint32_t*>(p);
+      }
+    }
 #pragma unroll
     for (int gi = 0; gi < GW; ++gi) {
       const int qg = GW * warp + gi;
@@ -340,8 +375,11 @@ __device__ __forceinline__ void attn_block(const AttnStage& st, float4 (*red)[4]
       const uint32_t wB = *reinterpret_cast<const uint32_t*>(vb + (cA + 1) * kAttnVStride) ^ 0x80808080u;
       const uint32_t wC = *reinterpret_cast<const uint32_t*>(vb + (cA + 8) * kAttnVStride) ^ 0x80808080u;
       const uint32_t wD = *reinterpret_cast<const uint32_t*>(vb + (cA + 9) * kAttnVStride) ^ 0x80808080u;
-      const __half2 sAB = __halves2half2(st.vs[cA * kNG + qg], st.vs[(cA + 1) * kNG + qg]);
-      const __half2 sCD = __halves2half2(st.vs[(cA + 8) * kNG + qg], st.vs[(cA + 9) * kNG + qg]);
+      const uint32_t hsel = (gi & 1) ? 0x7632u : 0x5410u;  // the group's fp16 of two cells' words
+      const uint32_t uAB = __byte_perm(vsw[0][gi >> 1], vsw[1][gi >> 1], hsel);
+      const uint32_t uCD = __byte_perm(vsw[2][gi >> 1], vsw[3][gi >> 1], hsel);
+      const __half2 sAB = *reinterpret_cast<const __half2*>(&uAB);
+      const __half2 sCD = *reinterpret_cast<const __half2*>(&uCD);
       // the two cells' bytes interleaved once: [A0 B0 A1 B1] and [A2 B2 A3 B3]
       const uint32_t ab[2] = {__byte_perm(wA, wB, 0x5140u), __byte_perm(wA, wB, 0x7362u)};
       const uint32_t cd[2] = {__byte_perm(wC, wD, 0x5140u), __byte_perm(wC, wD, 0x7362u)};
