@@ -9,14 +9,19 @@
 //    tensor cores instead of 6144 fp32 FMAs per gathered cell;
 //  * cells are gathered 32 at a time with cp.async (16-byte copies of whole
 //    256-byte K/V rows and their scales) into a double-buffered shared-memory
-//    ring, so the next block's gathers are in flight while one computes;
-//  * two warps split the 256 dims: each computes a partial QK^T over its 128
-//    dims (four scale groups), the two partials are summed through shared memory
-//    in a fixed order (both warps get bit-equal scores), each warp runs the same
-//    online softmax and accumulates P.V for its own 128 dims;
-//  * int8 codes become fp16 exactly (byte-permute with the 0x6400 exponent).  The
-//    per-32 K scale multiplies each 32-dim partial product in fp32 after the
-//    MMA; the per-32 V scale multiplies the fp16 V operand.  Q and P are fp16;
+//    ring, so the next block's gathers are in flight while one computes; each
+//    block's ids are loaded a block before its gathers are issued;
+//  * W warps split the 256 dims (W = 2 for prompt chunks, 4 for decode): each
+//    computes a partial QK^T over its dims, the partials are summed through shared
+//    memory in a fixed order (every warp gets bit-equal scores), each warp runs the
+//    same online softmax and accumulates P.V for its own dims;
+//  * int8 codes become fp16 exactly by byte-permute with the 0x6400 exponent, which
+//    gives 1152 + code.  For K the 1152 stays in: each 32-dim group's accumulator
+//    starts at -1152 times the group's sum of fp16 q, and the per-32 K scale
+//    multiplies the group's partial product in fp32 after the MMA.  For V the 1152
+//    is subtracted (the two cells of a B register interleaved by one byte-permute
+//    per four pairs) and the per-32 V scale multiplies the fp16 V operand.  Q and P
+//    are fp16, the weights 2^x from the hardware ex2;
 //  * the reference maximum of the online softmax moves only when a block
 //    exceeds it by more than 2^8, so P stays <= 256 and most blocks skip the
 //    rescale of O; split partials are reported against the true maximum;
