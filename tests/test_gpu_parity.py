@@ -406,6 +406,22 @@ def test_attn_prompt_kernel_golden(gpu):
         assert rel_err(out[r], want) <= OUT_TOL
 
 
+@pytest.mark.parametrize("rows,nsplit", [(3, 1), (3, 8), (12, 1)])
+def test_attn_query_offset(gpu, rows, nsplit):
+    # queries with a common offset of 2 standard deviations: the K codes enter the tiles as
+    # 1152 + code and each group's accumulator starts at -1152 times its query sum, so the
+    # cancellation is large here (both the decode and the prompt-chunk kernels).  Larger offsets
+    # take every variant past the tolerance through the fp16 rounding of q and P alone.
+    qsa = gpu
+    cells, k = 3000, 700
+    cache_h = synth.make_cache(241, cells)
+    q, _, _ = synth.make_queries(242, rows)
+    q = (q + 2.0).astype(np.float32)
+    q[0, 3] = -q[0, 3]  # one head with the opposite offset
+    ids = _id_lists(243, rows, cells, k, [k] * rows)
+    _check_attn(qsa, cache_h, qsa.DeviceCache.from_host(cache_h, DEV), q, ids, nsplit)
+
+
 def test_merge_vs_oracle(gpu):
     qsa = gpu
     st = synth.Stream(301, "merge")
