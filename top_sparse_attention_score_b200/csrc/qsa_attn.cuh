@@ -452,15 +452,16 @@ __global__ void __launch_bounds__(32 * W) attn_kernel(AttnArgs a) {
   AttnState<W> S;
   S.init();
   for (int b = 0; b < nblk; ++b) {
-    // refill the stage block b - 1 used (every warp finished it at the last barrier)
+    // block b has landed for every thread, and every warp has finished block b - 1 (its
+    // stage and the partial-score exchange are free again)
+    cp_async_wait<0>();
+    __syncthreads();
+    // refill the stage block b - 1 used
     const int nb = b + 1;
     if (nb < nblk) attn_gather<NT>(sm.st[nb % kAttnStages], a, kvh, static_cast<int>(threadIdx.x), ids);
     cp_async_commit();
     if (nb + 1 < nblk) load_ids(ids, nb + 1);
-    cp_async_wait<kAttnStages - 1>();
-    __syncthreads();
     attn_block<W>(sm.st[b % kAttnStages], sm.red, aq, kb, S, warp, [] { __syncthreads(); });
-    __syncthreads();
   }
   cp_async_wait<0>();
 
