@@ -148,3 +148,44 @@ def test_traffic_hash_follows_code_not_comments(tmp_path, monkeypatch):
     assert bench.source_hash("merge_kernel") == h0
     src.write_text(base.replace("x + 1", "x + 2"))
     assert bench.source_hash("merge_kernel") != h0
+
+
+def test_static_topk_status_and_trace_reject_bad_arguments(lib):
+    """The fixed-scratch selection's limits, the status read and the trace calls fail
+    with QSA_ERR_ARG before any CUDA call."""
+    from top_sparse_attention_score_b200 import qsa
+    P = ctypes.c_void_p(0x60000)
+    def static(ld=1024, rows=4, vis0=1000, top_k=64, scores=P, ids=P):
+        return lib.qsa_topk_static(scores, ld, rows, vis0, top_k, ids, None)
+    assert static(scores=None) == 1
+    assert static(ids=None) == 1
+    assert static(rows=0) == 1
+    assert static(rows=9) == 1 and "fixed scratch" in qsa.last_error()   # above QSA_STATIC_MAX_ROWS
+    assert static(top_k=0) == 1
+    assert static(top_k=2049) == 1 and "fixed scratch" in qsa.last_error()  # above QSA_STATIC_MAX_TOPK
+    assert static(vis0=0) == 1
+    assert static(vis0=1022) == 1                                 # row 3 sees 1025 > ld
+    assert static(ld=1026, vis0=100) == 1                         # ld % 4
+    assert static(ids=ctypes.c_void_p(0x60004)) == 1              # misaligned
+    assert lib.qsa_device_status(None, None) == 1
+    assert lib.qsa_trace_begin(0, None) == 1
+    assert lib.qsa_trace_begin(4097, None) == 1
+    n = ctypes.c_int(-1)
+    assert lib.qsa_trace_end(1, ctypes.byref(n), None, None) == 1 and "no trace" in qsa.last_error()
+
+
+def test_cache_and_chunk_limits(lib):
+    """A cache descriptor with misaligned arrays or an out-of-range size, and a prompt
+    chunk's top_k outside [1, QSA_MAX_TOPK], are rejected before any launch."""
+    from top_sparse_attention_score_b200 import qsa
+    P = ctypes.c_void_p(0x60000)
+    for cs in (qsa.CacheStruct(0x10008, 0x20000, 0x30000, 0x40000, 0x50000, 1000),  # misaligned k
+               qsa.CacheStruct(0x10000, 0x20000, 0x30000, 0x40000, 0x50000, 0),     # no cells
+               qsa.CacheStruct(0x10000, 0x20000, 0x30000, 0x40000, 0x50000, (1 << 24) + 1)):
+        assert lib.qsa_cache_write(ctypes.byref(cs), 0, 1, P, P, P, None) == 1
+        assert "cache" in qsa.last_error()
+    cb = ctypes.byref(_fake_cache(qsa))
+    for top_k in (0, 16385):
+        assert lib.qsa_prefill_chunk(cb, 0, 20, None, P, P, P, None, top_k, 0.0625, P, 1 << 40, P,
+                                     None, None) == 1
+        assert "top_k" in qsa.last_error()
